@@ -1,0 +1,191 @@
+// Skinny bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// out[m][n] (+)= s[n] * sum_k X[m][k] * W[n][k]      (fp32 accumulation in TMEM)
+//
+// The weight is the A operand (M = 128 output features per tile) and the activation is the
+// B operand (N = TN tokens), so a 63-token chunk fills one N = 64 tile and the weight
+// stream — the part that is HBM-bound at batch 1 — is split over many CTAs along N and K.
+// Split-K partial sums are added with fp32 reductions into an output that is either zero
+// (scratch, cleared by its consumer) or the fp32 residual stream itself (gated residual
+// "res + (x @ W) * gate" of the Realtime-VLA tech blog, kernel list "matmul_small_res_gate").
+//
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer and TMEM owner, warps 2..5 =
+// epilogue (TMEM -> registers -> global).  Every wait is bounded (DevCtl::timeout_ns).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rtvla {
+
+template <int TN>
+struct GemmCfg {
+  static constexpr int W_BYTES = 128 * 128;  // 128 rows x 64 bf16
+  static constexpr int X_BYTES = TN * 128;   // TN rows x 64 bf16
+  static constexpr int STAGE = W_BYTES + X_BYTES;
+  static constexpr int STAGES = (TN <= 64) ? 8 : (TN <= 128 ? 6 : 4);
+  static constexpr int TMEM_COLS = TN <= 32 ? 32 : (TN <= 64 ? 64 : (TN <= 128 ? 128 : 256));
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+};
+
+template <int TN>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, GemmParams p) {
+  using G = GemmCfg<TN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + G::STAGES * G::STAGE);
+  uint64_t *empty = full + G::STAGES;
+  uint64_t *done = empty + G::STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * 128;
+  const int m0 = blockIdx.y * TN;
+  const int kb_total = p.K >> 6;
+  const int kb0 = blockIdx.z * p.kb_per_split;
+  const int nkb = min(p.kb_per_split, kb_total - kb0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, G::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && nkb > 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % G::STAGES;
+        const uint32_t ph = (i / G::STAGES) & 1;
+        if (i >= G::STAGES && !mbar_wait(&empty[s], ph ^ 1, p.ctl, 101)) break;
+        uint8_t *st = smem + s * G::STAGE;
+        mbar_arrive_expect_tx(&full[s], G::STAGE);
+        tma_load_2d(st, &tmW, &full[s], (kb0 + i) * 64, p.w_row0 + n0, pol_w);
+        tma_load_2d(st + G::W_BYTES, &tmX, &full[s], (kb0 + i) * 64, m0, pol_x);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, TN);
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % G::STAGES;
+        const uint32_t ph = (i / G::STAGES) & 1;
+        if (!mbar_wait(&full[s], ph, p.ctl, 102)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + s * G::STAGE);
+        const uint32_t b = a + G::W_BYTES;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tmem, sdesc_k128(a + 32 * k), sdesc_k128(b + 32 * k), idesc, (i > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(done);
+    }
+  } else if (nkb > 0) {
+    // epilogue: warp (2..5) & 3 selects the TMEM lane quadrant it may access
+    const int q = warp & 3;
+    if (mbar_wait(done, 0, p.ctl, 103)) {
+      tc_fence_after();
+      const int n = n0 + q * 32 + lane;
+      const float sc = p.col_scale ? p.col_scale[n] : 1.0f;
+#pragma unroll 1
+      for (int c = 0; c < TN; c += 32) {
+        if (m0 + c >= p.M) break;
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int m = m0 + c + j;
+          if (m < p.M) {
+            float *o = p.out + (size_t)m * p.ldo + n;
+            if (p.atomic)
+              atomicAdd(o, v[j] * sc);
+            else
+              *o = v[j] * sc;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, G::TMEM_COLS);
+  }
+}
+
+template <int TN>
+static cudaError_t launch_tn(const CUtensorMap &tmW, const CUtensorMap &tmX, const GemmParams &p, int n_tiles,
+                             int m_tiles, int splits, cudaStream_t st) {
+  using G = GemmCfg<TN>;
+  dim3 grid(n_tiles, m_tiles, splits);
+  k_gemm_tc<TN><<<grid, 192, G::SMEM, st>>>(tmW, tmX, p);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_init_attributes() {
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<64>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<128>::SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tc<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<256>::SMEM);
+  return e;
+}
+
+// Chooses the token tile and the K split so that about one wave of 148 SMs is busy.
+GemmPlan gemm_plan(int M, int N, int K, int sm_count) {
+  GemmPlan g;
+  g.tn = (M <= 64) ? 64 : (M <= 1024 ? 128 : 256);
+  g.m_tiles = (M + g.tn - 1) / g.tn;
+  g.n_tiles = N / 128;
+  const int kb_total = K / 64;
+  const int units = g.n_tiles * g.m_tiles;
+  int splits = (sm_count + units - 1) / units;
+  if (splits < 1) splits = 1;
+  if (splits > kb_total) splits = kb_total;
+  g.kb_per_split = (kb_total + splits - 1) / splits;
+  g.splits = (kb_total + g.kb_per_split - 1) / g.kb_per_split;
+  return g;
+}
+
+int gemm_tile_index(int tn) { return tn <= 64 ? 0 : (tn <= 128 ? 1 : 2); }
+
+cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int M, int N, int K, float *out,
+                        int ldo, const float *col_scale, bool accumulate, DevCtl *ctl, int sm_count,
+                        cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  GemmPlan g = gemm_plan(M, N, K, sm_count);
+  GemmParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.w_row0 = w_row0;
+  p.kb_per_split = g.kb_per_split;
+  p.out = out;
+  p.ldo = ldo;
+  p.col_scale = col_scale;
+  p.atomic = (accumulate || g.splits > 1) ? 1 : 0;
+  p.ctl = ctl;
+  const CUtensorMap &tmX = xm.m[gemm_tile_index(g.tn)];
+  switch (g.tn) {
+    case 64: return launch_tn<64>(tmW, tmX, p, g.n_tiles, g.m_tiles, g.splits, st);
+    case 128: return launch_tn<128>(tmW, tmX, p, g.n_tiles, g.m_tiles, g.splits, st);
+    default: return launch_tn<256>(tmW, tmX, p, g.n_tiles, g.m_tiles, g.splits, st);
+  }
+}
+
+}  // namespace rtvla

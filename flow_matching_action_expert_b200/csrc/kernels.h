@@ -1,0 +1,97 @@
+// Host-side launchers of the rtvla kernels (internal to librtvla.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace rtvla {
+
+// ---------------------------------------------------------------------------------------
+// tcgen05 skinny GEMM
+struct GemmParams {
+  int M, N, K;
+  int w_row0;          // first row of this weight in the stacked tensor map
+  int kb_per_split;    // 64-wide K blocks per CTA
+  float *out;
+  int ldo;
+  const float *col_scale;  // per-output-column factor (AdaRMS gate) or null
+  int atomic;              // 1: fp32 reduction into out; 0: plain store
+  DevCtl *ctl;
+};
+
+struct GemmPlan {
+  int tn, m_tiles, n_tiles, splits, kb_per_split;
+};
+
+// One activation tensor map per token tile (box heights 64, 128, 256): the box must match
+// the tile the plan picks for the call's row count.
+struct XMaps {
+  CUtensorMap m[3];
+};
+int gemm_tile_index(int tn);
+GemmPlan gemm_plan(int M, int N, int K, int sm_count);
+cudaError_t gemm_init_attributes();
+
+// out[m][n] (+)= col_scale[n] * sum_k X[m][k] W[w_row0 + n][k].  `accumulate` adds into the
+// existing contents of out; otherwise out must be zero when the plan splits K.
+cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int M, int N, int K, float *out,
+                        int ldo, const float *col_scale, bool accumulate, DevCtl *ctl, int sm_count,
+                        cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------
+// attention (8 query heads share one KV head, head_dim 256)
+struct AttnParams {
+  const bf16 *q;            // [rows][q_ld], head h at column h*256; row = b*nq + i
+  int q_ld;
+  const CallArgs *ca;       // prefix K/V, valid lengths and cache stride of this call
+  int layer;
+  const bf16 *ksuf;         // suffix K/V [batch][n_suf][256] (may be null when n_suf = 0)
+  const bf16 *vsuf;
+  int n_suf;
+  int nq;                   // queries per sample
+  int keys_per_split;       // multiple of 64
+  int n_splits;
+  float *opart;             // [B][splits][nq][8][256] unnormalised partial outputs
+  float *mlpart;            // [B][splits][nq][8][2]   (running max in log2 units, sum)
+  bf16 *out;                // [rows][2048]
+  float scale_log2;         // log2(e) / sqrt(head_dim)
+  DevCtl *ctl;
+};
+
+cudaError_t attn_init_attributes();
+int attn_splits(int batch, int nq, int max_keys, int sm_count, int *keys_per_split);
+cudaError_t attn_launch(const AttnParams &p, int batch, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------
+// element-wise / row kernels
+cudaError_t launch_init_x(const CallArgs *ca, float *x, int n, cudaStream_t st);
+cudaError_t launch_action_in(const float *x, const bf16 *w_in, const float *b_in, float *h, int M,
+                             cudaStream_t st);
+cudaError_t launch_adanorm(const float *h, const float *s1p, bf16 *op, float *r, int M, float eps,
+                           cudaStream_t st);
+cudaError_t launch_qkv_post(float *acc, const float *r, const float *bias, const CallArgs *ca, int C,
+                            const float *rope_cos, const float *rope_sin, int rope_rows, bf16 *q, bf16 *ks,
+                            bf16 *vs, int M, DevCtl *ctl, cudaStream_t st);
+cudaError_t launch_gelu_mul(float *acc, const float *r, const float *bias, bf16 *out, int M, int F,
+                            cudaStream_t st);
+cudaError_t launch_final(const float *h, const float *s1p, const float *shift, const float *w_out,
+                         const float *b_out, float *x, int M, int final_norm, float eps, const CallArgs *ca,
+                         int write_actions, cudaStream_t st);
+// prefix pass
+cudaError_t launch_pf_mask(const CallArgs *ca, int B, int P, DevCtl *ctl, cudaStream_t st);
+cudaError_t launch_pf_embed(const CallArgs *ca, float *x, int M, int Dp, cudaStream_t st);
+cudaError_t launch_rmsnorm(const float *x, bf16 *op, int M, int Dp, float eps, cudaStream_t st);
+cudaError_t launch_pf_qkv_post(float *acc, const CallArgs *ca, int layer, int P, const float *rope_cos,
+                               const float *rope_sin, int rope_rows, bf16 *q, int M, DevCtl *ctl, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------
+// create-time precompute (fp64)
+cudaError_t launch_rows_dot_f64(const bf16 *W, int R, int Kd, const double *vecs, int S, const bf16 *bias,
+                                double *out, cudaStream_t st);
+cudaError_t launch_fold_cols(const bf16 *W, int R, int Kd, const bf16 *gamma, bf16 *out, cudaStream_t st);
+cudaError_t launch_scale_to_f32(const bf16 *w, int n, double s, float *out, cudaStream_t st);
+
+}  // namespace rtvla

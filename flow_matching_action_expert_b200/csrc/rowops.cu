@@ -1,0 +1,361 @@
+// Row-wise kernels of the denoise step and the prefix pass.
+//
+// Sources (Realtime-VLA tech blog): "Per-layer processing (PiGemmaDecoderLayer.forward)"
+// for the op order, kernel list entries "adarms_norm_style_proj" (RMS statistics, (1 +
+// scale) * x_norm + shift, gate kept apart), "matmul_rope_qkv" (RoPE applied to the QKV
+// output, three destinations Q/K/V) and "Scalar ops in GEMM epilogues" (token statistics
+// computed first, the normalisation factor applied after the GEMM accumulation).
+//
+// The AdaRMS of the expert is split accordingly: this file produces bf16(h * (1 + scale))
+// and r = rsqrt(mean(h^2) + eps); the GEMM consumer multiplies its accumulator by r and
+// adds shift @ W^T, a per-(step, layer) bias tabulated at create time.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rtvla {
+
+namespace {
+__device__ __forceinline__ float block_sum_256(float v, float *red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = (l < 8) ? red[l] : 0.f;
+  return warp_sum(s);
+}
+}  // namespace
+
+// x = noise (copy through the call's argument block)
+__global__ void k_init_x(const CallArgs *ca, float *x, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) x[i] = ca->noise[i];
+}
+
+// h[m][:] = x[m][:] @ W_in^T + b_in   (action_in_proj, 32 -> 1024)
+__global__ void __launch_bounds__(256) k_action_in(const float *x, const bf16 *w_in, const float *b_in, float *h) {
+  __shared__ float xs[32];
+  const int m = blockIdx.x;
+  if (threadIdx.x < 32) xs[threadIdx.x] = x[m * 32 + threadIdx.x];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int n = threadIdx.x + 256 * k;
+    const uint4 *wr = reinterpret_cast<const uint4 *>(w_in + n * 32);
+    float acc = b_in[n];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = wr[q];
+      const bf16 *e = reinterpret_cast<const bf16 *>(&v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc += bf2f(e[j]) * xs[q * 8 + j];
+    }
+    h[(size_t)m * 1024 + n] = acc;
+  }
+}
+
+// op = bf16(h * (1 + scale)), r = rsqrt(mean(h^2) + eps)   (width 1024)
+__global__ void __launch_bounds__(256) k_adanorm(const float *h, const float *s1p, bf16 *op, float *r, float eps) {
+  __shared__ float red[8];
+  const int m = blockIdx.x;
+  const float4 v = reinterpret_cast<const float4 *>(h + (size_t)m * 1024)[threadIdx.x];
+  const float ss = block_sum_256(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, red);
+  const float4 s = reinterpret_cast<const float4 *>(s1p)[threadIdx.x];
+  uint2 o;
+  o.x = pack_bf16(v.x * s.x, v.y * s.y);
+  o.y = pack_bf16(v.z * s.z, v.w * s.w);
+  reinterpret_cast<uint2 *>(op + (size_t)m * 1024)[threadIdx.x] = o;
+  if (threadIdx.x == 0) r[m] = rsqrtf(ss * (1.0f / 1024.0f) + eps);
+}
+
+// QKV epilogue: y = r * acc + bias; RoPE (pairs d, d+128) at position Lv_b + j on the 8 query
+// heads and the key; Q -> [M][2048], K_s, V_s -> [M][256] (bf16).  Clears acc.
+__global__ void __launch_bounds__(256) k_qkv_post(float *acc, const float *r, const float *bias, const CallArgs *ca,
+                                                  int C, const float *rc, const float *rs, int rope_rows, bf16 *q,
+                                                  bf16 *ks, bf16 *vs, DevCtl *ctl) {
+  const int m = blockIdx.x;
+  const int b = m / C, j = m % C;
+  int pos = ca->valid_len[b] + j;
+  if (pos < 0 || pos >= rope_rows) {
+    if (threadIdx.x == 0) set_error(ctl, DEVERR_BOUNDS, 301);
+    pos = pos < 0 ? 0 : rope_rows - 1;
+  }
+  float *a = acc + (size_t)m * 2560;
+  const float rr = r[m];
+  const float *cr = rc + (size_t)pos * 128;
+  const float *sr = rs + (size_t)pos * 128;
+  for (int i = threadIdx.x; i < 9 * 128; i += 256) {
+    const int head = i >> 7, d = i & 127;
+    const int c1 = head * 256 + d, c2 = c1 + 128;
+    const float x1 = rr * a[c1] + bias[c1];
+    const float x2 = rr * a[c2] + bias[c2];
+    const float co = cr[d], si = sr[d];
+    const float y1 = x1 * co - x2 * si;
+    const float y2 = x2 * co + x1 * si;
+    if (head < 8) {
+      q[(size_t)m * 2048 + c1] = f2bf(y1);
+      q[(size_t)m * 2048 + c2] = f2bf(y2);
+    } else {
+      ks[(size_t)m * 256 + d] = f2bf(y1);
+      ks[(size_t)m * 256 + d + 128] = f2bf(y2);
+    }
+  }
+  for (int d = threadIdx.x; d < 256; d += 256) vs[(size_t)m * 256 + d] = f2bf(rr * a[2304 + d] + bias[2304 + d]);
+  __syncthreads();
+  for (int i = threadIdx.x; i < 2560 / 4; i += 256) reinterpret_cast<float4 *>(a)[i] = make_float4(0, 0, 0, 0);
+}
+
+// out[m][j] = bf16(GELU_tanh(r*g + bg) * (r*u + bu)), g = acc[m][j], u = acc[m][F + j].  Clears acc.
+__global__ void __launch_bounds__(256) k_gelu_mul(float *acc, const float *r, const float *bias, bf16 *out, int F) {
+  const int m = blockIdx.x;
+  float *a = acc + (size_t)m * 2 * F;
+  const float rr = r ? r[m] : 1.0f;
+  for (int j = threadIdx.x * 4; j < F; j += 1024) {
+    float4 g = *reinterpret_cast<float4 *>(a + j);
+    float4 u = *reinterpret_cast<float4 *>(a + F + j);
+    float4 bg = make_float4(0, 0, 0, 0), bu = bg;
+    if (bias) {
+      bg = *reinterpret_cast<const float4 *>(bias + j);
+      bu = *reinterpret_cast<const float4 *>(bias + F + j);
+    }
+    uint2 o;
+    o.x = pack_bf16(gelu_tanh(rr * g.x + bg.x) * (rr * u.x + bu.x), gelu_tanh(rr * g.y + bg.y) * (rr * u.y + bu.y));
+    o.y = pack_bf16(gelu_tanh(rr * g.z + bg.z) * (rr * u.z + bu.z), gelu_tanh(rr * g.w + bg.w) * (rr * u.w + bu.w));
+    *reinterpret_cast<uint2 *>(out + (size_t)m * F + j) = o;
+    *reinterpret_cast<float4 *>(a + j) = make_float4(0, 0, 0, 0);
+    *reinterpret_cast<float4 *>(a + F + j) = make_float4(0, 0, 0, 0);
+  }
+}
+
+// Final AdaRMS (scale, shift) + action_out_proj with dt folded in + Euler:
+// x[m] += n @ (dt W_out)^T + dt b_out.  Writes the actions when asked.
+__global__ void __launch_bounds__(256) k_final(const float *h, const float *s1p, const float *shift, const float *w_out,
+                                               const float *b_out, float *x, int final_norm, float eps,
+                                               const CallArgs *ca, int write_actions) {
+  __shared__ float n[1024];
+  __shared__ float red[8];
+  const int m = blockIdx.x;
+  const float4 v = reinterpret_cast<const float4 *>(h + (size_t)m * 1024)[threadIdx.x];
+  const float ss = block_sum_256(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, red);
+  float4 y = v;
+  if (final_norm) {
+    const float r = rsqrtf(ss * (1.0f / 1024.0f) + eps);
+    const float4 s = reinterpret_cast<const float4 *>(s1p)[threadIdx.x];
+    const float4 t = reinterpret_cast<const float4 *>(shift)[threadIdx.x];
+    y = make_float4(r * v.x * s.x + t.x, r * v.y * s.y + t.y, r * v.z * s.z + t.z, r * v.w * s.w + t.w);
+  }
+  reinterpret_cast<float4 *>(n)[threadIdx.x] = y;
+  __syncthreads();
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int a = w * 4 + k;
+    const float *wr = w_out + a * 1024;
+    float acc = 0.f;
+    for (int d = l; d < 1024; d += 32) acc += n[d] * wr[d];
+    acc = warp_sum(acc);
+    if (l == 0) {
+      const float nx = x[m * 32 + a] + acc + b_out[a];
+      x[m * 32 + a] = nx;
+      if (write_actions) ca->actions[m * 32 + a] = nx;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// prefix pass
+
+// valid_len[b] = number of 1s in the pad mask; flags a mask whose valid tokens are not first.
+__global__ void k_pf_mask(const CallArgs *ca, int P, DevCtl *ctl) {
+  const int b = blockIdx.x;
+  const uint8_t *mk = ca->mask + (size_t)b * P;
+  int cnt = 0, bad = 0;
+  for (int j = threadIdx.x; j < P; j += blockDim.x) {
+    const int v = mk[j] != 0;
+    cnt += v;
+    if (v && j > 0 && mk[j - 1] == 0) bad = 1;
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  __shared__ int sc[32], sb[32];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) {
+    sc[w] = cnt;
+    sb[w] = bad;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int c = 0, bb = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+      c += sc[i];
+      bb |= sb[i];
+    }
+    ca->valid_out[b] = c;
+    if (bb) set_error(ctl, DEVERR_MASK, 401);
+  }
+}
+
+// x (fp32 residual) = embeddings
+__global__ void k_pf_embed(const CallArgs *ca, float *x, size_t n) {
+  const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (i >= n) return;
+  const uint4 v = *reinterpret_cast<const uint4 *>(ca->embeds + i);
+  const bf16 *e = reinterpret_cast<const bf16 *>(&v);
+  float4 *o = reinterpret_cast<float4 *>(x + i);
+  o[0] = make_float4(bf2f(e[0]), bf2f(e[1]), bf2f(e[2]), bf2f(e[3]));
+  o[1] = make_float4(bf2f(e[4]), bf2f(e[5]), bf2f(e[6]), bf2f(e[7]));
+}
+
+// op = bf16(x * rsqrt(mean(x^2) + eps)); the RMSNorm weight (1 + w) is folded into the next GEMM.
+__global__ void __launch_bounds__(256) k_rmsnorm(const float *x, bf16 *op, int Dp, float eps) {
+  __shared__ float red[8];
+  const int m = blockIdx.x;
+  const float *xr = x + (size_t)m * Dp;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 4; i < Dp; i += 1024) {
+    const float4 v = *reinterpret_cast<const float4 *>(xr + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = block_sum_256(ss, red);
+  const float r = rsqrtf(ss / (float)Dp + eps);
+  for (int i = threadIdx.x * 4; i < Dp; i += 1024) {
+    const float4 v = *reinterpret_cast<const float4 *>(xr + i);
+    uint2 o;
+    o.x = pack_bf16(v.x * r, v.y * r);
+    o.y = pack_bf16(v.z * r, v.w * r);
+    *reinterpret_cast<uint2 *>(op + (size_t)m * Dp + i) = o;
+  }
+}
+
+// Prefill QKV epilogue: RoPE at position j (the valid tokens come first, so cumsum(mask) - 1
+// = j on them); Q -> q, K and V -> the output cache of this layer.  Clears acc.
+__global__ void __launch_bounds__(256) k_pf_qkv_post(float *acc, const CallArgs *ca, int layer, int P,
+                                                     const float *rc, const float *rs, int rope_rows, bf16 *q,
+                                                     DevCtl *ctl) {
+  const int m = blockIdx.x;
+  const int b = m / P, j = m % P;
+  int pos = j;
+  if (pos >= rope_rows) {
+    if (threadIdx.x == 0) set_error(ctl, DEVERR_BOUNDS, 302);
+    pos = rope_rows - 1;
+  }
+  float *a = acc + (size_t)m * 2560;
+  const size_t kvo = (((size_t)layer * ca->batch + b) * ca->cap + j) * 256;
+  const float *cr = rc + (size_t)pos * 128;
+  const float *sr = rs + (size_t)pos * 128;
+  for (int i = threadIdx.x; i < 9 * 128; i += 256) {
+    const int head = i >> 7, d = i & 127;
+    const int c1 = head * 256 + d, c2 = c1 + 128;
+    const float x1 = a[c1], x2 = a[c2];
+    const float co = cr[d], si = sr[d];
+    const float y1 = x1 * co - x2 * si, y2 = x2 * co + x1 * si;
+    if (head < 8) {
+      q[(size_t)m * 2048 + c1] = f2bf(y1);
+      q[(size_t)m * 2048 + c2] = f2bf(y2);
+    } else {
+      ca->kvo_k[kvo + d] = f2bf(y1);
+      ca->kvo_k[kvo + d + 128] = f2bf(y2);
+    }
+  }
+  for (int d = threadIdx.x; d < 256; d += 256) ca->kvo_v[kvo + d] = f2bf(a[2304 + d]);
+  __syncthreads();
+  for (int i = threadIdx.x; i < 2560 / 4; i += 256) reinterpret_cast<float4 *>(a)[i] = make_float4(0, 0, 0, 0);
+}
+
+// ---------------------------------------------------------------------------------------
+// create-time precompute in fp64
+
+// out[s][r] = sum_k W[r][k] * vecs[s][k] + bias[r]  (one warp per row r, S <= 64)
+__global__ void k_rows_dot_f64(const bf16 *W, int R, int Kd, const double *vecs, int S, const bf16 *bias,
+                               double *out) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int l = threadIdx.x & 31;
+  if (r >= R) return;
+  const bf16 *wr = W + (size_t)r * Kd;
+  for (int s = 0; s < S; ++s) {
+    const double *v = vecs + (size_t)s * Kd;
+    double acc = 0.0;
+    for (int k = l; k < Kd; k += 32) acc += (double)bf2f(wr[k]) * v[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (l == 0) out[(size_t)s * R + r] = acc + (bias ? (double)bf2f(bias[r]) : 0.0);
+  }
+}
+
+// out[r][k] = bf16(W[r][k] * (1 + gamma[k]))  (Gemma RMSNorm weight folded into the next Linear)
+__global__ void k_fold_cols(const bf16 *W, int R, int Kd, const bf16 *gamma, bf16 *out) {
+  const size_t n = (size_t)R * Kd;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int k = (int)(i % Kd);
+    out[i] = f2bf(bf2f(W[i]) * (1.0f + bf2f(gamma[k])));
+  }
+}
+
+__global__ void k_scale_to_f32(const bf16 *w, int n, double s, float *out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = (float)((double)bf2f(w[i]) * s);
+}
+
+// ---------------------------------------------------------------------------------------
+// launchers
+cudaError_t launch_init_x(const CallArgs *ca, float *x, int n, cudaStream_t st) {
+  k_init_x<<<(n + 255) / 256, 256, 0, st>>>(ca, x, n);
+  return cudaGetLastError();
+}
+cudaError_t launch_action_in(const float *x, const bf16 *w_in, const float *b_in, float *h, int M, cudaStream_t st) {
+  k_action_in<<<M, 256, 0, st>>>(x, w_in, b_in, h);
+  return cudaGetLastError();
+}
+cudaError_t launch_adanorm(const float *h, const float *s1p, bf16 *op, float *r, int M, float eps, cudaStream_t st) {
+  k_adanorm<<<M, 256, 0, st>>>(h, s1p, op, r, eps);
+  return cudaGetLastError();
+}
+cudaError_t launch_qkv_post(float *acc, const float *r, const float *bias, const CallArgs *ca, int C,
+                            const float *rope_cos, const float *rope_sin, int rope_rows, bf16 *q, bf16 *ks,
+                            bf16 *vs, int M, DevCtl *ctl, cudaStream_t st) {
+  k_qkv_post<<<M, 256, 0, st>>>(acc, r, bias, ca, C, rope_cos, rope_sin, rope_rows, q, ks, vs, ctl);
+  return cudaGetLastError();
+}
+cudaError_t launch_gelu_mul(float *acc, const float *r, const float *bias, bf16 *out, int M, int F, cudaStream_t st) {
+  k_gelu_mul<<<M, 256, 0, st>>>(acc, r, bias, out, F);
+  return cudaGetLastError();
+}
+cudaError_t launch_final(const float *h, const float *s1p, const float *shift, const float *w_out, const float *b_out,
+                         float *x, int M, int final_norm, float eps, const CallArgs *ca, int write_actions,
+                         cudaStream_t st) {
+  k_final<<<M, 256, 0, st>>>(h, s1p, shift, w_out, b_out, x, final_norm, eps, ca, write_actions);
+  return cudaGetLastError();
+}
+cudaError_t launch_pf_mask(const CallArgs *ca, int B, int P, DevCtl *ctl, cudaStream_t st) {
+  k_pf_mask<<<B, 256, 0, st>>>(ca, P, ctl);
+  return cudaGetLastError();
+}
+cudaError_t launch_pf_embed(const CallArgs *ca, float *x, int M, int Dp, cudaStream_t st) {
+  const size_t n = (size_t)M * Dp;
+  k_pf_embed<<<(unsigned)((n / 8 + 255) / 256), 256, 0, st>>>(ca, x, n);
+  return cudaGetLastError();
+}
+cudaError_t launch_rmsnorm(const float *x, bf16 *op, int M, int Dp, float eps, cudaStream_t st) {
+  k_rmsnorm<<<M, 256, 0, st>>>(x, op, Dp, eps);
+  return cudaGetLastError();
+}
+cudaError_t launch_pf_qkv_post(float *acc, const CallArgs *ca, int layer, int P, const float *rope_cos,
+                               const float *rope_sin, int rope_rows, bf16 *q, int M, DevCtl *ctl, cudaStream_t st) {
+  k_pf_qkv_post<<<M, 256, 0, st>>>(acc, ca, layer, P, rope_cos, rope_sin, rope_rows, q, ctl);
+  return cudaGetLastError();
+}
+cudaError_t launch_rows_dot_f64(const bf16 *W, int R, int Kd, const double *vecs, int S, const bf16 *bias,
+                                double *out, cudaStream_t st) {
+  k_rows_dot_f64<<<(R + 7) / 8, 256, 0, st>>>(W, R, Kd, vecs, S, bias, out);
+  return cudaGetLastError();
+}
+cudaError_t launch_fold_cols(const bf16 *W, int R, int Kd, const bf16 *gamma, bf16 *out, cudaStream_t st) {
+  k_fold_cols<<<1184, 256, 0, st>>>(W, R, Kd, gamma, out);
+  return cudaGetLastError();
+}
+cudaError_t launch_scale_to_f32(const bf16 *w, int n, double s, float *out, cudaStream_t st) {
+  k_scale_to_f32<<<(n + 255) / 256, 256, 0, st>>>(w, n, s, out);
+  return cudaGetLastError();
+}
+
+}  // namespace rtvla

@@ -1,0 +1,222 @@
+/*
+ * rtvla.h — C ABI of librtvla.so: the π0.5 action-expert flow-matching denoise loop and the
+ * Gemma-2B-shaped prefix pass that fills its KV cache, as hand-written CUDA for sm_100a.
+ *
+ * What the calls compute is defined by:
+ *   [BLOG]  Realtime-VLA tech blog (blog.w4k4.me): "pi0.5 inference flow" (encoder phase run
+ *           once, then a 10-step denoise loop), "Inference branch structure" (encoder-only
+ *           and decoder-only branches of PaliGemmaWithExpertModel.forward), "Per-layer
+ *           processing (PiGemmaDecoderLayer.forward)", "Precompute (__init__)", "CUDA Graph"
+ *           (inputs copied in, one replay) and "Static buffers".
+ *   [PAPER] "Running VLAs at Real-time Speed" (arXiv 2510.26742), Sec. 3.1-3.2, Table 1.
+ *
+ * Conventions for every call:
+ *   - All tensors are row-major and contiguous.  Weight matrices use the (out, in) layout of
+ *     a Linear layer: element [o][i] multiplies input i into output o.  "bf16" is IEEE
+ *     bfloat16 (uint16 storage); "f32" is IEEE float.
+ *   - Pointers named *device* must point to memory of the CUDA device that was current when
+ *     rtvla_create ran; pointers named *host* are ordinary CPU memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously unless the call says otherwise.
+ *   - Argument and shape errors are returned synchronously, before anything is enqueued.
+ *     Errors the GPU detects (a bounded wait that expired, an index out of range, a pad mask
+ *     that is not a prefix) set a device error word that rtvla_sync_status reports.  Nothing
+ *     aborts, traps or throws across the ABI.
+ *   - One context serves one stream at a time: calls on one context must not overlap on the
+ *     GPU (they share the context's static activation buffers).
+ */
+#ifndef RTVLA_H
+#define RTVLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct rtvla_ctx rtvla_ctx; /* opaque; owned by the library */
+
+typedef enum {
+  RTVLA_OK = 0,
+  RTVLA_ERR_INVALID_ARG = 1,     /* null pointer, negative size, bad enum value */
+  RTVLA_ERR_SHAPE = 2,           /* batch / prefix length / chunk beyond the context's capacity */
+  RTVLA_ERR_MASK_NOT_PREFIX = 3, /* pad mask has a valid token after a padded one (device-detected) */
+  RTVLA_ERR_OOM = 4,             /* cudaMalloc failed while creating the context */
+  RTVLA_ERR_CUDA = 5,            /* a CUDA runtime call failed; the context may be unusable */
+  RTVLA_ERR_DEVICE_TIMEOUT = 6,  /* a bounded device-side wait expired (device-detected) */
+  RTVLA_ERR_UNSUPPORTED = 7,     /* model shape the kernels are not built for */
+  RTVLA_ERR_DEVICE_BOUNDS = 8    /* a valid length exceeded its buffer (device-detected, clamped) */
+} rtvla_status;
+
+/* Engines that run the denoise loop (rtvla_config.engine). */
+enum {
+  RTVLA_ENGINE_AUTO = 0,       /* persistent kernel when it applies, else layered */
+  RTVLA_ENGINE_LAYERED = 1,    /* one kernel per phase, the whole loop captured as one CUDA graph */
+  RTVLA_ENGINE_PERSISTENT = 2  /* one persistent kernel per call that streams weights continuously */
+};
+
+/*
+ * Model and capacity description.  The kernels are built for the π0.5 shapes of [BLOG
+ * "pi0.5 inference flow"]: width 1024, MLP 4096, 8 query heads x 256, 1 KV head, action
+ * dim 32 (expert); width 2048, MLP 16384, 8 x 256, 1 KV head (prefix pass).  Other values
+ * return RTVLA_ERR_UNSUPPORTED.  n_layers and n_steps are free (1..64 and 1..64).
+ */
+typedef struct {
+  int n_layers;    /* expert layers L (18; 2 for the tiny expert); the prefix pass has as many */
+  int width;       /* D = 1024 */
+  int mlp_dim;     /* F = 4096 */
+  int n_q_heads;   /* 8 */
+  int n_kv_heads;  /* 1 */
+  int head_dim;    /* 256 */
+  int action_dim;  /* 32 */
+  int chunk;       /* C, actions per chunk (1..256) */
+  int n_steps;     /* Euler steps S (10); t_k = 1 - k/S, dt = -1/S */
+  int max_prefix;  /* capacity P_max of the prefix KV cache in tokens (>= 1) */
+  int max_batch;   /* largest batch any call will use (>= 1) */
+  int final_norm;  /* 1: AdaRMS before action_out_proj; 0: none */
+  int has_prefill; /* 1: also build the prefix pass (needs the pf_* weights) */
+  int pf_width;    /* 2048 when has_prefill */
+  int pf_mlp_dim;  /* 16384 when has_prefill */
+  int engine;      /* RTVLA_ENGINE_* */
+  float rms_eps;   /* 1e-6 */
+  float rope_theta;/* 10000 */
+} rtvla_config;
+
+/*
+ * Weights: device pointers to bf16 tensors in (out, in) layout, owned by the caller and
+ * read only during rtvla_create (the library keeps its own folded copies, so the caller
+ * may free these when rtvla_create returns).  Per-layer fields are host arrays of
+ * n_layers device pointers.
+ */
+typedef struct {
+  const void *action_in_w;  /* [D][A]  action_in_proj */
+  const void *action_in_b;  /* [D] */
+  const void *action_out_w; /* [A][D]  action_out_proj */
+  const void *action_out_b; /* [A] */
+  const void *time_in_w;    /* [D][D]  time_mlp_in */
+  const void *time_in_b;    /* [D] */
+  const void *time_out_w;   /* [D][D]  time_mlp_out */
+  const void *time_out_b;   /* [D] */
+  const void *const *wq;    /* [L] -> [H*hd][D] */
+  const void *const *wk;    /* [L] -> [hd][D] */
+  const void *const *wv;    /* [L] -> [hd][D] */
+  const void *const *wo;    /* [L] -> [D][H*hd] */
+  const void *const *wg;    /* [L] -> [F][D]  gate_proj */
+  const void *const *wu;    /* [L] -> [F][D]  up_proj */
+  const void *const *wd;    /* [L] -> [D][F]  down_proj */
+  const void *const *ada_attn_w; /* [L] -> [3D][D]  input_layernorm dense (scale|shift|gate) */
+  const void *const *ada_attn_b; /* [L] -> [3D] */
+  const void *const *ada_ffn_w;  /* [L] -> [3D][D]  post_attention_layernorm dense */
+  const void *const *ada_ffn_b;  /* [L] -> [3D] */
+  const void *ada_final_w;  /* [3D][D]  final norm dense (used when final_norm = 1) */
+  const void *ada_final_b;  /* [3D] */
+  /* prefix pass (has_prefill = 1): Gemma RMSNorm weights w (scale 1 + w) and projections */
+  const void *const *pf_ln1; /* [L] -> [Dp] */
+  const void *const *pf_wq;  /* [L] -> [H*hd][Dp] */
+  const void *const *pf_wk;  /* [L] -> [hd][Dp] */
+  const void *const *pf_wv;  /* [L] -> [hd][Dp] */
+  const void *const *pf_wo;  /* [L] -> [Dp][H*hd] */
+  const void *const *pf_ln2; /* [L] -> [Dp] */
+  const void *const *pf_wg;  /* [L] -> [Fp][Dp] */
+  const void *const *pf_wu;  /* [L] -> [Fp][Dp] */
+  const void *const *pf_wd;  /* [L] -> [Dp][Fp] */
+} rtvla_weights;
+
+/*
+ * Prefix KV cache (caller-owned device memory).  [BLOG "pi0.5 inference flow", encoder
+ * step 4: past_key_values of every layer].  K is stored after RoPE ("rotate half" pairs
+ * (d, d+128), position p of prefix token p).  Only tokens [0, valid_len[b]) of sample b are
+ * read; the rest may hold anything.
+ */
+typedef struct {
+  void *k;             /* device bf16 [n_layers][batch][prefix_cap][head_dim] */
+  void *v;             /* device bf16 [n_layers][batch][prefix_cap][head_dim] */
+  int32_t *valid_len;  /* device int32 [batch], each in [0, prefix_cap] */
+  int batch;           /* 1..max_batch */
+  int prefix_cap;      /* 1..max_prefix, the token stride of k and v */
+} rtvla_kv;
+
+/*
+ * Creates a context: repacks and folds the weights and builds the per-step tables of
+ * [BLOG "Precompute (__init__)"] — time embedding and time MLP for the S fixed timesteps,
+ * every AdaRMS dense output (scale, shift, gate) for every (step, layer), Q/K/V
+ * concatenated, dt folded into action_out_proj, RoPE cos/sin — and allocates every
+ * activation buffer once [BLOG "Static buffers"].  Synchronous.  On success *out owns
+ * device memory until rtvla_destroy.  Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA.
+ */
+rtvla_status rtvla_create(const rtvla_weights *w, const rtvla_config *cfg, rtvla_ctx **out);
+
+/* Bytes of K plus V for a cache of `batch` samples x `prefix_cap` tokens (0 on bad args). */
+size_t rtvla_kv_bytes(const rtvla_config *cfg, int batch, int prefix_cap);
+
+/*
+ * Prefix pass [BLOG "pi0.5 inference flow", encoder steps 3-4; "Inference branch
+ * structure", encoder-only branch].  prefix_embeds: device bf16 [batch][prefix_len][pf_width],
+ * already scaled by sqrt(2048).  pad_mask: device uint8 [batch][prefix_len], 1 = valid; the
+ * valid tokens of each sample must come first.  Fills kv_out->k / kv_out->v for every layer
+ * (rows >= the valid length hold unspecified values) and kv_out->valid_len.  The last layer
+ * computes K/V only.  Errors: INVALID_ARG, SHAPE (batch > max_batch, prefix_len >
+ * kv_out->prefix_cap or > max_prefix), UNSUPPORTED (no prefill built); device-detected
+ * MASK_NOT_PREFIX through rtvla_sync_status.
+ */
+rtvla_status rtvla_prefill(rtvla_ctx *ctx, const void *prefix_embeds, const uint8_t *pad_mask,
+                           int batch, int prefix_len, const rtvla_kv *kv_out, void *stream);
+
+/*
+ * The denoise loop [BLOG "pi0.5 inference flow", decoder phase steps 1-4; "Inference
+ * branch structure", decoder-only branch]: x = noise at t = 1; for k = 0..S-1 the expert
+ * predicts v_t from x, the prefix KV and t_k = 1 - k/S, and x += dt * v_t with dt = -1/S.
+ * noise, actions_out: device f32 [kv->batch][chunk][action_dim] (may alias).  Runs as one
+ * CUDA-graph replay or one persistent launch on `stream`.  Errors: INVALID_ARG, SHAPE;
+ * device-detected DEVICE_TIMEOUT / DEVICE_BOUNDS through rtvla_sync_status.
+ */
+rtvla_status rtvla_sample_actions(rtvla_ctx *ctx, const float *noise, const rtvla_kv *kv,
+                                  float *actions_out, void *stream);
+
+/*
+ * Same loop from host buffers: copies noise (host f32 [batch][chunk][action_dim]), the
+ * cache (host bf16 k and v [n_layers][batch][prefix_cap][head_dim], host int32 valid_len
+ * [batch]) to the context's device staging, runs the loop, copies the actions back to
+ * actions_out (host f32) and waits for the stream.  Host buffers should be pinned for full
+ * copy speed.  The staging cache is allocated on first use (RTVLA_ERR_OOM on failure).
+ */
+rtvla_status rtvla_sample_actions_host(rtvla_ctx *ctx, const float *noise, const void *kv_k,
+                                       const void *kv_v, const int32_t *valid_len, int batch,
+                                       int prefix_cap, float *actions_out, void *stream);
+
+/*
+ * Waits for `stream`, then reads and clears the device error word: RTVLA_OK, or the first
+ * device-detected error (DEVICE_TIMEOUT, DEVICE_BOUNDS, MASK_NOT_PREFIX) since the last call.
+ */
+rtvla_status rtvla_sync_status(rtvla_ctx *ctx, void *stream);
+
+/*
+ * Test hook: runs the loop up to and including step `step` (0-based) with the layered
+ * engine and writes the expert hidden state of that step before layer 0 and after each
+ * layer to h_layers: device f32 [n_layers + 1][batch][chunk][width].  Asynchronous.
+ */
+rtvla_status rtvla_debug_trace(rtvla_ctx *ctx, const float *noise, const rtvla_kv *kv, int step,
+                               float *h_layers, void *stream);
+
+/* Number of kernels of this library one rtvla_sample_actions call launches at `batch`
+ * with the context's engine (after the call has been made once at that batch). */
+int rtvla_kernels_per_call(rtvla_ctx *ctx, int batch);
+
+/* Selects the engine for later calls (RTVLA_ENGINE_*); INVALID_ARG on a bad value. */
+rtvla_status rtvla_set_engine(rtvla_ctx *ctx, int engine);
+
+/* Bounded device waits give up after this many microseconds (default 2,000,000). */
+rtvla_status rtvla_set_wait_timeout_us(rtvla_ctx *ctx, long long us);
+
+/* Frees everything the context owns (waits for the device first).  NULL is a no-op. */
+void rtvla_destroy(rtvla_ctx *ctx);
+
+/* Static English text for a status code. */
+const char *rtvla_status_string(rtvla_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTVLA_H */

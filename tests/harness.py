@@ -1,0 +1,125 @@
+"""Shared helpers of the GPU tests: seeded workloads onto the device, calls through the C ABI
+binding, and the comparison metrics with the tolerances of the parity contract."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import flow_matching_action_expert_b200 as R
+from synth import gen
+from synth import workloads as WL
+
+# tolerances: actions max-abs 3e-2 and relative L2 1e-2; per-layer hidden states (and their
+# per-layer updates) relative L2 1e-2; prefix KV relative L2 1e-2 on the valid rows
+ACT_MAX_ABS = 3e-2
+ACT_REL_L2 = 1e-2
+H_REL_L2 = 1e-2
+KV_REL_L2 = 1e-2
+
+
+def rel_l2(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def bf16_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bf16_host_f32(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy()
+
+
+class GpuModel:
+    """One rtvla context built from seeded bf16 weights."""
+
+    def __init__(self, wl: WL.Workload, expert_bits: dict, prefill_bits: dict | None = None,
+                 max_batch: int | None = None, max_prefix: int | None = None, engine: int = R.ENGINE_AUTO,
+                 final_norm: bool | None = None):
+        dev = {k: bf16_dev(v) for k, v in expert_bits.items()}
+        if prefill_bits is not None:
+            dev.update({k: bf16_dev(v) for k, v in prefill_bits.items()})
+        s = wl.expert
+        self.cfg = R.make_config(n_layers=s.n_layers, chunk=wl.chunk, max_prefix=max_prefix or wl.prefix_cap,
+                                 max_batch=max_batch or wl.batch, n_steps=s.n_steps,
+                                 final_norm=s.final_norm if final_norm is None else final_norm,
+                                 has_prefill=prefill_bits is not None, engine=engine)
+        self.ctx = R.rtvla_create(dev, self.cfg)
+        del dev
+        torch.cuda.synchronize()
+        self.wl = wl
+
+    def close(self):
+        if self.ctx:
+            R.rtvla_destroy(self.ctx)
+            self.ctx = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def kv(self, k: torch.Tensor, v: torch.Tensor, valid: torch.Tensor, batch: int, cap: int):
+        return R.make_kv(k, v, valid, batch, cap)
+
+    def sample(self, noise: np.ndarray, k: torch.Tensor, v: torch.Tensor, valid: torch.Tensor) -> np.ndarray:
+        B, C, A = noise.shape
+        cap = k.shape[2]
+        x = torch.from_numpy(np.ascontiguousarray(noise, dtype=np.float32)).cuda()
+        out = torch.empty_like(x)
+        R.rtvla_sample_actions(self.ctx, x, self.kv(k, v, valid, B, cap), out)
+        st = R.rtvla_sync_status(self.ctx)
+        assert st == 0, R.STATUS[st]
+        return out.cpu().numpy()
+
+    def trace(self, noise: np.ndarray, k, v, valid, step: int) -> np.ndarray:
+        B, C, A = noise.shape
+        cap = k.shape[2]
+        x = torch.from_numpy(np.ascontiguousarray(noise, dtype=np.float32)).cuda()
+        L = self.cfg.n_layers
+        h = torch.empty((L + 1, B, C, 1024), dtype=torch.float32, device="cuda")
+        R.rtvla_debug_trace(self.ctx, x, self.kv(k, v, valid, B, cap), step, h)
+        st = R.rtvla_sync_status(self.ctx)
+        assert st == 0, R.STATUS[st]
+        return h.cpu().numpy()
+
+    def prefill(self, emb_bits: np.ndarray, mask: np.ndarray, cap: int | None = None):
+        B, P, _ = emb_bits.shape
+        cap = cap or P
+        L = self.cfg.n_layers
+        k = torch.zeros((L, B, cap, 256), dtype=torch.bfloat16, device="cuda")
+        v = torch.zeros_like(k)
+        valid = torch.zeros(B, dtype=torch.int32, device="cuda")
+        e = bf16_dev(emb_bits)
+        m = torch.from_numpy(np.ascontiguousarray(mask)).cuda()
+        R.rtvla_prefill(self.ctx, e, m, B, P, R.make_kv(k, v, valid, B, cap))
+        return k, v, valid
+
+
+def device_kv(wl: WL.Workload, pad_fill: float | None = None):
+    kb, vb, valid = WL.kv_cache(wl, pad_fill=pad_fill)
+    return (bf16_dev(kb), bf16_dev(vb), torch.from_numpy(valid).cuda(),
+            gen.bf16_to_f32(kb), gen.bf16_to_f32(vb), valid)
+
+
+def assert_actions_close(gpu, ref, what=""):
+    d = float(np.abs(gpu - ref).max())
+    r = rel_l2(gpu, ref)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite actions"
+    assert d <= ACT_MAX_ABS and r <= ACT_REL_L2, f"{what}: max-abs {d:.3e} rel-L2 {r:.3e}"
+    return d, r
+
+
+def assert_trace_close(gpu_tr, ref_tr, what=""):
+    worst = 0.0
+    for i in range(ref_tr.shape[0]):
+        r = rel_l2(gpu_tr[i], ref_tr[i])
+        worst = max(worst, r)
+        assert r <= H_REL_L2, f"{what}: hidden state {i} rel-L2 {r:.3e}"
+        if i > 0:
+            dr = rel_l2(gpu_tr[i] - gpu_tr[i - 1], ref_tr[i] - ref_tr[i - 1])
+            worst = max(worst, dr)
+            assert dr <= H_REL_L2, f"{what}: layer {i - 1} update rel-L2 {dr:.3e}"
+    return worst
