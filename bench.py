@@ -1,0 +1,337 @@
+"""Benchmark of the π0.5 action-expert 10-step denoise loop (2-view: 512-token prefix KV
+cache, chunk 63, batch 1, 18 layers) through the rtvla C ABI.
+
+One step = one full 10-step denoise loop (one rtvla_sample_actions call) on inputs already
+resident in HBM.  Prints one JSON line (rank 0).  Multi-GPU runs are independent replicas
+(the method does not shard); the timed region is bracketed by a barrier and a device
+synchronize, and the time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--batch B]
+
+--impl reference times the fp64 CPU oracle (plain numpy) on the host cores: each step is
+one Euler step of the same workload (the oracle with S = 1), reported per 10-step loop.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "10-step denoise latency ms (2-view, chunk 63); achieved HBM GB/s vs roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--batch", type=int, default=1)
+    p.add_argument("--engine", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-flush", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def workload(batch):
+    from synth import workloads as WL
+    return WL.workload(3) if batch == 1 else WL.workload(4, batch=batch)
+
+
+def algorithmic(wl):
+    """Bytes and FLOPs one 10-step loop must move / execute (weights streamed every step,
+    valid prefix KV read, per-step tables, suffix K/V written and read)."""
+    s = wl.expert
+    L, D, F, H, hd, A, S = s.n_layers, s.width, s.mlp_dim, s.n_q_heads, s.head_dim, s.action_dim, s.n_steps
+    per_layer_params = (H * hd + 2 * hd) * D + D * H * hd + 2 * F * D + D * F
+    params = L * per_layer_params + 2 * D * A
+    M = wl.batch * wl.chunk
+    lv = sum(wl.valid_lens)
+    w_bytes = params * 2
+    kv_bytes = L * lv * hd * 2 * 2
+    table_bytes = L * (4 * D + (H * hd + 2 * hd) + 2 * F) * 4
+    suffix_bytes = L * M * hd * 2 * 2 * 2
+    bytes_step = w_bytes + kv_bytes + table_bytes + suffix_bytes
+    attn_flops = sum(4 * H * wl.chunk * (l + wl.chunk) * hd for l in wl.valid_lens) * L
+    flops_step = 2 * M * params + attn_flops
+    return bytes_step * S, flops_step * S, w_bytes * S
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.rows = []
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                self.rows.append(f)
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_one_step_ms(wl, steps):
+    """Times the fp64 oracle on one Euler step (S = 1) of the workload, `steps` times."""
+    from dataclasses import replace
+
+    from oracle import model as O
+    from synth import gen
+    from synth import workloads as WL
+    bits = WL.expert_weights(wl.expert)
+    W = O.Weights(WL.as_f32(bits))
+    kb, vb, valid = WL.kv_cache(wl)
+    kf, vf = gen.bf16_to_f32(kb), gen.bf16_to_f32(vb)
+    noise = WL.noise(wl)
+    one = replace(wl.expert, n_steps=1)
+    O.sample_actions(W, one, noise[:1], kf[:, :1], vf[:, :1], valid[:1])  # widen weights once (not timed)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        O.sample_actions(W, one, noise, kf, vf, valid)
+        times.append((time.perf_counter() - t0) * 1e3)
+    return times
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    wl = workload(args.batch)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state beyond widening the weights (done once, untimed)
+    times = oracle_one_step_ms(wl, max(1, args.steps))
+    per_loop = statistics.mean(times) * wl.expert.n_steps
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(per_loop, 3), "unit": "ms",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_loop, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,0.02) bf16 weights, N(0,1) KV and noise)",
+        "config": {"workload": wl.name, "batch": wl.batch, "chunk": wl.chunk, "prefix": wl.prefix_cap,
+                   "layers": wl.expert.n_layers, "steps_per_loop": wl.expert.n_steps},
+        "cpu_baseline": {"value": round(per_loop, 3), "unit": "ms", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"{len(times)} x one Euler step of the loop (fp64 oracle, S=1), x10 per loop"},
+        "e2e": {"value": round(per_loop, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import flow_matching_action_expert_b200 as R
+    from synth import workloads as WL
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workload(args.batch)
+    bits = WL.expert_weights(wl.expert)
+    dw = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev) for k, v in bits.items()}
+    cfg = R.make_config(n_layers=wl.expert.n_layers, chunk=wl.chunk, max_prefix=wl.prefix_cap,
+                        max_batch=wl.batch, engine=args.engine)
+    ctx = R.rtvla_create(dw, cfg)
+    del dw
+    kb, vb, valid = WL.kv_cache(wl)
+    noise_np = WL.noise(wl)
+    k = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).to(dev)
+    v = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16).to(dev)
+    vl = torch.from_numpy(valid).to(dev)
+    noise = torch.from_numpy(noise_np).to(dev)
+    out = torch.empty_like(noise)
+    kv = R.make_kv(k, v, vl, wl.batch, wl.prefix_cap)
+    stream = torch.cuda.current_stream(dev)
+    flush = None if args.no_flush else torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def call():
+        R.rtvla_sample_actions(ctx, noise, kv, out, stream)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    st = R.rtvla_sync_status(ctx, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {R.STATUS[st]}")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local_rank) as clk:
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(float(i))          # L2 flush (256 MiB write) outside the timed events
+            starts[i].record(stream)
+            call()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = statistics.mean(per)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    st = R.rtvla_sync_status(ctx, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {R.STATUS[st]}")
+    kernels = R.rtvla_kernels_per_call(ctx, wl.batch)
+
+    # end to end through the host-buffer entry point (pinned noise + KV in, actions out)
+    hk = torch.from_numpy(kb.view(np.int16)).pin_memory()
+    hv = torch.from_numpy(vb.view(np.int16)).pin_memory()
+    hl = torch.from_numpy(valid).pin_memory()
+    hn = torch.from_numpy(noise_np).pin_memory()
+    ho = torch.empty_like(hn).pin_memory()
+    for _ in range(2):
+        R.rtvla_sample_actions_host(ctx, hn, hk, hv, hl, wl.batch, wl.prefix_cap, ho, stream)
+    e2e = []
+    for i in range(args.steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        R.rtvla_sample_actions_host(ctx, hn, hk, hv, hl, wl.batch, wl.prefix_cap, ho, stream)
+        e1.record(stream)
+        e1.synchronize()
+        e2e.append(e0.elapsed_time(e1))
+    e2e_ms = statistics.mean(e2e)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = hn.numel() * 4 + hk.numel() * 2 + hv.numel() * 2 + hl.numel() * 4
+    d2h = ho.numel() * 4
+    R.rtvla_destroy(ctx)
+
+    if rank != 0:
+        return
+    hbm, bf16_pk, bf16_sus, src = peaks()
+    bytes_loop, flops_loop, w_bytes = algorithmic(wl)
+    achieved_gbs = bytes_loop / (ms * 1e-3) / 1e9
+    achieved_tf = flops_loop / (ms * 1e-3) / 1e12
+    t_mem = bytes_loop / (hbm * 1e9)
+    t_tc = flops_loop / (bf16_sus * 1e12)
+    bound = "hbm" if t_mem >= t_tc else "tensor"
+    engine = {0: "auto", 1: "layered", 2: "persistent"}[args.engine]
+    line = {
+        "metric": METRIC, "value": round(ms, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) bf16 weights, N(0,1) KV and noise)",
+        "config": {"workload": wl.name, "batch": wl.batch, "chunk": wl.chunk, "prefix": wl.prefix_cap,
+                   "valid_prefix": list(wl.valid_lens)[:4], "layers": wl.expert.n_layers,
+                   "steps_per_loop": wl.expert.n_steps, "engine": engine, "parallelism": f"replicas{world}",
+                   "l2": ("flushed by a 256 MiB write between timed loops; weights (623 MB) exceed L2"
+                          if flush is not None else "not flushed; weights (623 MB) exceed L2")},
+        "hbm_gbs_achieved": round(achieved_gbs, 1),
+        "chunks_per_s": round(world * wl.batch / (ms * 1e-3), 2),
+        "latency_ms": {"p10": round(float(np.percentile(per, 10)), 4), "p50": round(float(np.median(per)), 4),
+                       "p90": round(float(np.percentile(per, 90)), 4)},
+        "roofline": {"bound": bound, "kernel": f"rtvla_sample_actions ({engine} engine, one call)",
+                     "achieved": round(achieved_gbs if bound == "hbm" else achieved_tf, 1),
+                     "peak": hbm if bound == "hbm" else bf16_sus,
+                     "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                     "frac": round((achieved_gbs / hbm) if bound == "hbm" else (achieved_tf / bf16_sus), 4),
+                     "traffic": None, "peak_source": src,
+                     "algorithmic_bytes_per_launch": int(bytes_loop), "algorithmic_flops_per_launch": int(flops_loop),
+                     "roofline_ms": round(max(t_mem, t_tc) * 1e3, 4)},
+        "e2e": {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(kernels * args.steps) if kernels > 0 else None,
+        "kernels_per_step": kernels,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        times = oracle_one_step_ms(wl, 3)
+        per_loop = statistics.mean(times) * wl.expert.n_steps
+        line["cpu_baseline"] = {"value": round(per_loop, 1), "unit": "ms", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": "3 x one Euler step of the same workload (fp64 oracle, S=1), x10 per loop"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
