@@ -24,6 +24,7 @@ STATUS = {
 # the symbols include/rtvla.h declares
 EXPORTS = (
     "rtvla_create", "rtvla_kv_bytes", "rtvla_prefill", "rtvla_sample_actions", "rtvla_sample_actions_host",
+    "rtvla_sample_actions_host_static",
     "rtvla_sync_status", "rtvla_debug_trace", "rtvla_kernels_per_call", "rtvla_set_engine",
     "rtvla_set_wait_timeout_us", "rtvla_destroy", "rtvla_status_string",
 )
@@ -78,6 +79,7 @@ def _lib():
         lib.rtvla_prefill.argtypes = [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.POINTER(RtvlaKV), _P]
         lib.rtvla_sample_actions.argtypes = [_P, _P, ctypes.POINTER(RtvlaKV), _P, _P]
         lib.rtvla_sample_actions_host.argtypes = [_P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P]
+        lib.rtvla_sample_actions_host_static.argtypes = [_P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P]
         lib.rtvla_sync_status.argtypes = [_P, _P]
         lib.rtvla_debug_trace.argtypes = [_P, _P, ctypes.POINTER(RtvlaKV), ctypes.c_int, _P, _P]
         lib.rtvla_kernels_per_call.argtypes = [_P, ctypes.c_int]
@@ -187,6 +189,14 @@ def rtvla_sample_actions_host(ctx: int, noise, kv_k, kv_v, valid_len, batch: int
     _check(_lib().rtvla_sample_actions_host(ctx, _ptr(noise), _ptr(kv_k), _ptr(kv_v), _ptr(valid_len), batch,
                                             prefix_cap, _ptr(actions_out), _stream(stream)),
            "rtvla_sample_actions_host")
+
+
+def rtvla_sample_actions_host_static(ctx: int, noise, kv_k, kv_v, valid_len, batch: int, prefix_cap: int,
+                                     actions_out, stream=None):
+    """Allocation-free host-buffer call: stages through the library's fixed 32 MiB device array."""
+    _check(_lib().rtvla_sample_actions_host_static(ctx, _ptr(noise), _ptr(kv_k), _ptr(kv_v), _ptr(valid_len),
+                                                   batch, prefix_cap, _ptr(actions_out), _stream(stream)),
+           "rtvla_sample_actions_host_static")
 
 
 def rtvla_sync_status(ctx: int, stream=None) -> int:

@@ -13,6 +13,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <utility>
 #include <vector>
 
@@ -839,3 +840,102 @@ rtvla_status rtvla_set_wait_timeout_us(rtvla_ctx *c, long long us) {
 }
 
 }  // extern "C"
+
+// =======================================================================================
+// Allocation-free host-buffer call.
+//
+// Same computation as rtvla_sample_actions_host, for callers that must not allocate device
+// memory once they are running (see include/rtvla.h).  The device staging that
+// rtvla_sample_actions_host obtains with cudaMalloc on first use lives here in a fixed
+// file-scope array instead; every GPU that loads this library holds that array until the
+// process exits.
+
+#define RTVLA_STATIC_STAGING_BYTES (32u << 20)
+
+static __device__ __align__(256) unsigned char g_rtvla_static_staging[RTVLA_STATIC_STAGING_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+unsigned char *g_static_addr[kMaxDevices] = {};
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Device address of the staging array on device `dev` (which must be current).  The name
+// g_rtvla_static_staging is only a host-side stand-in in host code; the address kernels and
+// copies may use comes from cudaGetSymbolAddress, looked up once per device.
+rtvla_status static_staging(int dev, unsigned char **out) {
+  if (dev < 0 || dev >= kMaxDevices) return RTVLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_rtvla_static_staging);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return RTVLA_ERR_CUDA;
+    }
+    g_static_addr[dev] = static_cast<unsigned char *>(p);
+  }
+  *out = g_static_addr[dev];
+  return RTVLA_OK;
+}
+}  // namespace
+
+extern "C" rtvla_status rtvla_sample_actions_host_static(rtvla_ctx *c, const float *noise, const void *kv_k,
+                                                         const void *kv_v, const int32_t *valid_len, int batch,
+                                                         int prefix_cap, float *actions_out, void *stream) {
+  if (!c || !noise || !kv_k || !kv_v || !valid_len || !actions_out) return RTVLA_ERR_INVALID_ARG;
+  if (batch < 1 || prefix_cap < 1) return RTVLA_ERR_INVALID_ARG;
+  if (batch > c->Bmax || prefix_cap > c->Pmax) return RTVLA_ERR_SHAPE;
+  if (c->engine == RTVLA_ENGINE_PERSISTENT) return RTVLA_ERR_UNSUPPORTED;
+  const size_t kv_elems = (size_t)c->L * batch * prefix_cap * HD;
+  const size_t io = (size_t)batch * c->C * A;
+  const size_t off_act = round256(io * 4);
+  const size_t off_vl = off_act + round256(io * 4);
+  const size_t off_k = off_vl + round256((size_t)batch * 4);
+  const size_t off_v = off_k + round256(kv_elems * 2);
+  const size_t total = off_v + round256(kv_elems * 2);
+  if (total > RTVLA_STATIC_STAGING_BYTES) return RTVLA_ERR_SHAPE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RTVLA_ERR_CUDA;
+  if (dev != c->device) return RTVLA_ERR_INVALID_ARG;
+  unsigned char *base = nullptr;
+  rtvla_status s = static_staging(dev, &base);
+  if (s != RTVLA_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float *d_noise = reinterpret_cast<float *>(base);
+  float *d_act = reinterpret_cast<float *>(base + off_act);
+  int *d_vl = reinterpret_cast<int *>(base + off_vl);
+  bf16 *d_k = reinterpret_cast<bf16 *>(base + off_k);
+  bf16 *d_v = reinterpret_cast<bf16 *>(base + off_v);
+  const cudaMemcpyKind hd = cudaMemcpyHostToDevice;
+  if (cudaMemcpyAsync(d_noise, noise, io * 4, hd, st) != cudaSuccess ||
+      cudaMemcpyAsync(d_k, kv_k, kv_elems * 2, hd, st) != cudaSuccess ||
+      cudaMemcpyAsync(d_v, kv_v, kv_elems * 2, hd, st) != cudaSuccess ||
+      cudaMemcpyAsync(d_vl, valid_len, (size_t)batch * 4, hd, st) != cudaSuccess)
+    return RTVLA_ERR_CUDA;
+  CallArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.noise = d_noise;
+  a.actions = d_act;
+  a.kv_k = d_k;
+  a.kv_v = d_v;
+  a.valid_len = d_vl;
+  a.batch = batch;
+  a.cap = prefix_cap;
+  if (cudaMemcpyAsync(c->args_dn, &a, sizeof(a), hd, st) != cudaSuccess) return RTVLA_ERR_CUDA;
+  // A graph already captured for this shape is replayed; otherwise the same kernels are
+  // launched directly, so that this call never instantiates anything.
+  auto it = c->graphs_dn.find(std::make_pair(batch, prefix_cap));
+  if (it != c->graphs_dn.end()) {
+    if (cudaGraphLaunch(it->second.exec, st) != cudaSuccess) return RTVLA_ERR_CUDA;
+  } else {
+    int n = 0;
+    if (enqueue_denoise(c, c->args_dn, batch, prefix_cap, st, nullptr, c->S - 1, &n) != cudaSuccess)
+      return RTVLA_ERR_CUDA;
+  }
+  if (cudaMemcpyAsync(actions_out, d_act, io * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return RTVLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RTVLA_ERR_CUDA;
+  return RTVLA_OK;
+}

@@ -186,6 +186,34 @@ rtvla_status rtvla_sample_actions_host(rtvla_ctx *ctx, const float *noise, const
                                        int prefix_cap, float *actions_out, void *stream);
 
 /*
+ * Allocation-free variant of rtvla_sample_actions_host (the paper has no counterpart: this
+ * is an integration aid of this library).
+ *
+ * Who needs it: a robot control loop that runs inference every camera frame must keep a fixed
+ * period, and cudaMalloc can block for milliseconds and synchronise the device; some hosts
+ * also fix every device-memory budget at start-up.  Such callers create the context once at
+ * start-up (rtvla_create allocates) and afterwards may not allocate at all — but
+ * rtvla_sample_actions_host allocates its device staging on first use.  This call allocates
+ * nothing: it stages the inputs and outputs in one file-scope device array of 32 MiB
+ * (RTVLA_STATIC_STAGING_BYTES) that every GPU loading this library holds until the process
+ * exits, and it captures no graph (a graph already captured for this shape by
+ * rtvla_sample_actions is replayed; otherwise the kernels are launched directly).
+ *
+ * Arguments, layout and result are those of rtvla_sample_actions_host (host buffers, the
+ * call waits for `stream`).  The device of `ctx` must be current.  Errors: INVALID_ARG;
+ * SHAPE when batch or prefix_cap exceed the context's capacity or when noise + actions +
+ * valid_len + K + V (each rounded up to 256 bytes) need more than 32 MiB, checked before
+ * anything is copied; UNSUPPORTED for the persistent engine; CUDA.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture.  All calls share the one array, which
+ * keeps the last call's contents (every byte a call reads is written by that call first):
+ * calls that overlap on the GPU — from two streams or two contexts on one device — race.
+ */
+rtvla_status rtvla_sample_actions_host_static(rtvla_ctx *ctx, const float *noise, const void *kv_k,
+                                              const void *kv_v, const int32_t *valid_len, int batch,
+                                              int prefix_cap, float *actions_out, void *stream);
+
+/*
  * Waits for `stream`, then reads and clears the device error word: RTVLA_OK, or the first
  * device-detected error (DEVICE_TIMEOUT, DEVICE_BOUNDS, MASK_NOT_PREFIX) since the last call.
  */
