@@ -20,8 +20,6 @@ struct DevCtl {
   int err;                       // OR of DEVERR_*
   int where;                     // first failing site (diagnostic)
   unsigned long long timeout_ns; // limit of every bounded wait
-  unsigned int bar_count;        // grid barrier arrival counter (persistent engine)
-  unsigned int bar_gen;          // grid barrier generation
 };
 
 // Per-call pointers, written to device memory before each graph replay / persistent launch
@@ -40,6 +38,9 @@ struct CallArgs {
   bf16 *kvo_v;
   int *valid_out;
   int pf_len;           // prefill tokens per sample
+  // persistent engine: grid-barrier arrival counters, 8 of them 128 bytes apart (all 0 in every
+  // copy from the host)
+  alignas(128) unsigned int bar_count[8 * 32];
 };
 
 __device__ __forceinline__ void set_error(DevCtl *ctl, int code, int where) {
@@ -76,6 +77,15 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
   return 0.5f * x * (1.0f + tanhf(k0 * (x + 0.044715f * x * x * x)));
+}
+
+// GELU, tanh approximation, with the hardware tanh (tanh.approx.f32, relative error about
+// 2^-11, below the bf16 rounding of the result)
+__device__ __forceinline__ float gelu_tanh_fast(float x) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(k0 * (x + 0.044715f * x * x * x)));
+  return 0.5f * x * (1.0f + t);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -135,6 +145,18 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16)
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
@@ -147,6 +169,26 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uin
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+
+// Bulk tensor reduce-add: global[tile at (x, y)] += shared tile, performed by the TMA unit
+// (one request per tile instead of one atomic per element).  x * 4 must be a multiple of 16.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *m, const void *src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared source of every committed bulk operation has been read
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed bulk operation has completed its global writes
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------------------

@@ -1,0 +1,51 @@
+// Persistent engine of the denoise loop (one cooperative kernel per call; batch 1, chunk <= 64).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace rtvla {
+
+struct PersistParams {
+  const CallArgs *ca;       // noise, actions, prefix cache, valid length
+  unsigned int *bar;        // grid-barrier counter (zeroed by the per-call argument copy)
+  int L, S, C;
+  int final_norm;
+  float eps;
+  float scale_log2;         // log2(e) / sqrt(head_dim)
+  int attn_splits, attn_kps;
+  // folded weights and per-(step, layer) tables (library-owned)
+  const bf16 *w_in;
+  const float *b_in, *w_out, *b_out;
+  const float *s1p_attn, *gate_attn, *s1p_ffn, *gate_ffn, *bias_qkv, *bias_gu, *s1p_fin, *shift_fin;
+  const float *rope_cos, *rope_sin;
+  // activations (library-owned static buffers)
+  float *x, *h, *acc_qkv, *acc_gu, *ss_attn, *ss_ffn, *opart, *mlpart;
+  bf16 *o;                  // attention output [64][2048] (O-projection operand)
+  bf16 *qb, *ks, *vs;       // finalised Q [64][2048], suffix K / V [64][256]
+  DevCtl *ctl;
+  // optional phase timestamps (globaltimer ns), [grid][max_phases][8]: 0 phase start,
+  // 1 operand ready, 2 accumulator ready, 3 epilogue issued, 4 attention queries staged,
+  // 5 first key chunk staged, 6 attention done, 7 barrier arrival; null unless the
+  // environment variable RTVLA_PHASE_STAMPS names the file rtvla_destroy writes them to
+  unsigned long long *stamps;
+  int max_phases;
+};
+
+int persistent_smem_bytes();
+cudaError_t persistent_init_attributes();
+bool persistent_fits(int sm_count);
+void persistent_attn_plan(int keys, int sm_count, int *splits, int *kps);
+int persistent_max_splits(int sm_count);  // upper bound of the splits any plan returns
+// Tensor maps of the persistent kernel.
+struct PersistMaps {
+  CUtensorMap w_qkv, w_o, w_gu, w_d;  // stacked bf16 weights, 64-column x 128-row boxes, 128B swizzle
+  CUtensorMap r_qkv, r_gu, r_h;       // fp32 bulk-reduce targets acc_qkv, acc_gu, h (128 x 64 boxes)
+  CUtensorMap l_h, l_gu;              // fp32 loads of h and acc_gu, 32-column x 64-row boxes, 128B swizzle
+  CUtensorMap l_o;                    // bf16 load of the attention output, 64 x 64 boxes, 128B swizzle
+};
+cudaError_t persistent_launch(const PersistMaps &m, const PersistParams &p, int grid, cudaStream_t st);
+
+}  // namespace rtvla

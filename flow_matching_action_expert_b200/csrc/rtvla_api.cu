@@ -10,6 +10,8 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstddef>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <map>
@@ -19,6 +21,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "persistent.h"
 #include "rtvla.h"
 
 using namespace rtvla;
@@ -56,10 +59,16 @@ struct rtvla_ctx {
   int Mpmax = 0;
   float *px = nullptr, *pacc = nullptr, *popart = nullptr, *pmlpart = nullptr;
   bf16 *pop = nullptr, *pq = nullptr, *po = nullptr, *pmb = nullptr;
+  // persistent engine
+  bool pers_ok = false;
+  float *ss_attn = nullptr, *ss_ffn = nullptr, *pk_opart = nullptr, *pk_mlpart = nullptr;
+  unsigned long long *pk_stamps = nullptr;
+  int pk_max_phases = 0;
   // control
   DevCtl *ctl = nullptr;
   CallArgs *args_dn = nullptr, *args_pf = nullptr, *args_tr = nullptr;
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_pwqkv, tm_pwo, tm_pwgu, tm_pwd;
+  PersistMaps pmaps;                // tensor maps of the persistent engine
   XMaps tm_op, tm_o, tm_mb, tm_pop, tm_po, tm_pmb;
   std::map<std::pair<int, int>, GraphEntry> graphs_dn, graphs_pf;
   std::map<int, int> kernels_per_call;
@@ -96,6 +105,19 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, ui
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// fp32 [rows][cols] row-major; box = box_cols x 64 rows.  128-column boxes without swizzle
+// are bulk-reduce targets; 32-column boxes with 128-byte swizzle are staging loads.
+bool make_map_f32(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols, bool swz) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {box_cols, 64};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -300,6 +322,56 @@ rtvla_status capture(rtvla_ctx *c, bool prefill, int B, int P, GraphEntry *out) 
   out->exec = ex;
   out->kernels = n;
   return RTVLA_OK;
+}
+
+bool use_persistent(const rtvla_ctx *c, int batch) {
+  if (c->engine == RTVLA_ENGINE_LAYERED) return false;
+  return c->pers_ok && batch == 1;
+}
+
+cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, int cap, cudaStream_t st) {
+  PersistParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.ca = dargs;
+  p.bar = reinterpret_cast<unsigned int *>(reinterpret_cast<char *>(dargs) + offsetof(CallArgs, bar_count));
+  static_assert(offsetof(CallArgs, bar_count) % 128 == 0, "barrier counters must start a 128-byte line");
+  p.L = c->L;
+  p.S = c->S;
+  p.C = c->C;
+  p.final_norm = c->cfg.final_norm;
+  p.eps = c->cfg.rms_eps;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
+  persistent_attn_plan(cap + c->C, c->sm_count, &p.attn_splits, &p.attn_kps);
+  p.w_in = c->w_in;
+  p.b_in = c->b_in;
+  p.w_out = c->w_out;
+  p.b_out = c->b_out;
+  p.s1p_attn = c->s1p_attn;
+  p.gate_attn = c->gate_attn;
+  p.s1p_ffn = c->s1p_ffn;
+  p.gate_ffn = c->gate_ffn;
+  p.bias_qkv = c->bias_qkv;
+  p.bias_gu = c->bias_gu;
+  p.s1p_fin = c->s1p_fin;
+  p.shift_fin = c->shift_fin;
+  p.rope_cos = c->rope_cos;
+  p.rope_sin = c->rope_sin;
+  p.x = c->x;
+  p.h = c->h;
+  p.acc_qkv = c->acc_qkv;
+  p.acc_gu = c->acc_gu;
+  p.ss_attn = c->ss_attn;
+  p.ss_ffn = c->ss_ffn;
+  p.opart = c->pk_opart;
+  p.mlpart = c->pk_mlpart;
+  p.o = c->o;
+  p.qb = c->q;
+  p.ks = c->ks;
+  p.vs = c->vs;
+  p.ctl = c->ctl;
+  p.stamps = c->pk_stamps;
+  p.max_phases = c->pk_max_phases;
+  return persistent_launch(c->pmaps, p, c->sm_count, st);
 }
 
 rtvla_status build_tables(rtvla_ctx *c, const rtvla_weights *w) {
@@ -580,6 +652,34 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
   }
   if (!ok) return RTVLA_ERR_CUDA;
 
+  // ---- persistent engine (batch 1, chunk <= 64): norm statistics and attention partials
+  if (persistent_init_attributes() != cudaSuccess) return RTVLA_ERR_CUDA;
+  c->pers_ok = C <= 64 && persistent_fits(c->sm_count);
+  if (c->pers_ok) {
+    const int sp = persistent_max_splits(c->sm_count);
+    c->ss_attn = dalloc<float>(c, 64);
+    c->ss_ffn = dalloc<float>(c, 64);
+    c->pk_opart = dalloc<float>(c, (size_t)sp * NQH * 64 * HD);
+    c->pk_mlpart = dalloc<float>(c, (size_t)sp * NQH * 64 * 2);
+    if (!c->ss_attn || !c->ss_ffn || !c->pk_opart || !c->pk_mlpart) return RTVLA_ERR_OOM;
+    PersistMaps &pm = c->pmaps;
+    pm.w_qkv = c->tm_wqkv;
+    pm.w_o = c->tm_wo;
+    pm.w_gu = c->tm_wgu;
+    pm.w_d = c->tm_wd;
+    pm.l_o = c->tm_o.m[0];
+    if (!make_map_f32(&pm.r_qkv, c->acc_qkv, 64, 2560, 128, false) ||
+        !make_map_f32(&pm.r_gu, c->acc_gu, 64, 2 * F, 128, false) || !make_map_f32(&pm.r_h, c->h, 64, D, 128, false) ||
+        !make_map_f32(&pm.l_h, c->h, 64, D, 32, true) || !make_map_f32(&pm.l_gu, c->acc_gu, 64, 2 * F, 32, true))
+      return RTVLA_ERR_CUDA;
+    if (std::getenv("RTVLA_PHASE_STAMPS")) {
+      c->pk_max_phases = c->S * (7 * c->L + 1) + 2;
+      c->pk_stamps = dalloc<unsigned long long>(c, (size_t)c->sm_count * c->pk_max_phases * 8);
+      if (!c->pk_stamps) return RTVLA_ERR_OOM;
+      cudaMemset(c->pk_stamps, 0, (size_t)c->sm_count * c->pk_max_phases * 8 * 8);
+    }
+  }
+
   // ---- control block and argument blocks
   c->ctl = dalloc<DevCtl>(c, 1);
   c->args_dn = dalloc<CallArgs>(c, 1);
@@ -652,6 +752,20 @@ rtvla_status rtvla_create(const rtvla_weights *w, const rtvla_config *cfg, rtvla
 void rtvla_destroy(rtvla_ctx *c) {
   if (!c) return;
   cudaDeviceSynchronize();
+  if (c->pk_stamps) {
+    // debug aid: raw phase timestamps of the last persistent launch, [grid][phases][8] u64
+    const char *path = std::getenv("RTVLA_PHASE_STAMPS");
+    const size_t n = (size_t)c->sm_count * c->pk_max_phases * 8;
+    std::vector<unsigned long long> h(n);
+    if (path && cudaMemcpy(h.data(), c->pk_stamps, n * 8, cudaMemcpyDeviceToHost) == cudaSuccess) {
+      if (FILE *f = std::fopen(path, "wb")) {
+        const int hdr[2] = {c->sm_count, c->pk_max_phases};
+        std::fwrite(hdr, sizeof(hdr), 1, f);
+        std::fwrite(h.data(), 8, n, f);
+        std::fclose(f);
+      }
+    }
+  }
   free_all(c);
 }
 
@@ -682,7 +796,16 @@ rtvla_status rtvla_sample_actions(rtvla_ctx *c, const float *noise, const rtvla_
   CallArgs a = host_args(kv);
   a.noise = noise;
   a.actions = actions_out;
-  if (c->engine == RTVLA_ENGINE_PERSISTENT) return RTVLA_ERR_UNSUPPORTED;
+  if (c->engine == RTVLA_ENGINE_PERSISTENT && !use_persistent(c, kv->batch)) return RTVLA_ERR_UNSUPPORTED;
+  if (use_persistent(c, kv->batch)) {
+    if (cudaMemcpyAsync(c->args_dn, &a, sizeof(a), cudaMemcpyHostToDevice, st) != cudaSuccess) return RTVLA_ERR_CUDA;
+    if (launch_persistent(c, c->args_dn, kv->prefix_cap, st) != cudaSuccess) {
+      cudaGetLastError();
+      return RTVLA_ERR_CUDA;
+    }
+    c->kernels_per_call[kv->batch] = 1;
+    return RTVLA_OK;
+  }
   const auto key = std::make_pair(kv->batch, kv->prefix_cap);
   auto it = c->graphs_dn.find(key);
   if (it == c->graphs_dn.end()) {

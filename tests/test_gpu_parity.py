@@ -26,6 +26,9 @@ def _oracle(wl, wf, kf, vf, valid, noise, trace_step=None, batch_indices=None):
                             batch_indices=batch_indices)
 
 
+ENGINES = {"layered": R.ENGINE_LAYERED, "persistent": R.ENGINE_PERSISTENT}
+
+
 @pytest.mark.parametrize("variant", ["plain", "stressed", "biased"])
 def test_tiny_expert_actions_and_layers(variant):
     wl = WL.workload(1)
@@ -36,20 +39,23 @@ def test_tiny_expert_actions_and_layers(variant):
     k, v, valid, kf, vf, vnp = device_kv(wl)
     noise = WL.noise(wl)
     ref, rtr0 = _oracle(wl, wf, kf, vf, vnp, noise, trace_step=0)
-    out = m.sample(noise, k, v, valid)
-    assert_actions_close(out, ref, f"tiny/{variant}")
+    for name, eng in ENGINES.items():
+        R.rtvla_set_engine(m.ctx, eng)
+        out = m.sample(noise, k, v, valid)
+        assert_actions_close(out, ref, f"tiny/{variant}/{name}")
     assert_trace_close(m.trace(noise, k, v, valid, 0), rtr0[:, :], f"tiny/{variant} step 0")
     _, rtr9 = _oracle(wl, wf, kf, vf, vnp, noise, trace_step=9)
     assert_trace_close(m.trace(noise, k, v, valid, 9), rtr9, f"tiny/{variant} step 9")
     m.close()
 
 
+@pytest.mark.parametrize("engine", sorted(ENGINES))
 @pytest.mark.parametrize("cfg", [2, 3])
-def test_full_expert_actions(cfg):
+def test_full_expert_actions(cfg, engine):
     wl = WL.workload(cfg)
     bits = WL.expert_weights(wl.expert)
     wf = WL.as_f32(bits)
-    m = GpuModel(wl, bits)
+    m = GpuModel(wl, bits, engine=ENGINES[engine])
     k, v, valid, kf, vf, vnp = device_kv(wl)
     noise = WL.noise(wl)
     ref, rtr = _oracle(wl, wf, kf, vf, vnp, noise, trace_step=4)
@@ -97,6 +103,41 @@ def test_edge_cases_lengths_chunks_and_padding():
         out = m.sample(noise, k, v, valid)
         assert_actions_close(out, ref, wl.name)
         m.close()
+
+
+def test_persistent_engine_edge_cases():
+    base = WL.workload(1)
+    bits = WL.expert_weights(base.expert, stressed=True)
+    wf = WL.as_f32(bits)
+    for chunk, lv in ((1, 0), (64, 130), (37, 1), (64, 0)):
+        wl = WL.Workload(f"edge B1 C{chunk} Lv{lv}", base.expert, chunk, 1, 130, (lv,))
+        m = GpuModel(wl, bits, engine=R.ENGINE_PERSISTENT)
+        k, v, valid, kf, vf, vnp = device_kv(wl, pad_fill=3.0e4)
+        noise = WL.noise(wl)
+        ref = _oracle(wl, wf, kf, vf, vnp, noise)
+        out = m.sample(noise, k, v, valid)
+        assert_actions_close(out, ref, wl.name)
+        assert R.rtvla_kernels_per_call(m.ctx, 1) == 1
+        m.close()
+
+
+def test_bounded_waits_report_a_timeout_and_the_context_recovers():
+    wl = WL.workload(1)
+    bits = WL.expert_weights(wl.expert)
+    wf = WL.as_f32(bits)
+    m = GpuModel(wl, bits, engine=R.ENGINE_PERSISTENT)
+    k, v, valid, kf, vf, vnp = device_kv(wl)
+    noise_np = WL.noise(wl)
+    noise = torch.from_numpy(noise_np).cuda()
+    out = torch.empty_like(noise)
+    kv = R.make_kv(k, v, valid, 1, wl.prefix_cap)
+    R.rtvla_set_wait_timeout_us(m.ctx, 1)          # every grid barrier gives up after 1 us
+    R.rtvla_sample_actions(m.ctx, noise, kv, out)
+    assert R.STATUS[R.rtvla_sync_status(m.ctx)] == "RTVLA_ERR_DEVICE_TIMEOUT"
+    R.rtvla_set_wait_timeout_us(m.ctx, 2_000_000)
+    got = m.sample(noise_np, k, v, valid)
+    assert_actions_close(got, _oracle(wl, wf, kf, vf, vnp, noise_np), "after timeout")
+    m.close()
 
 
 def test_host_buffer_entry_point_matches_device_entry_point():
