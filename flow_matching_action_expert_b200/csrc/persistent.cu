@@ -29,11 +29,11 @@ namespace pk {
 
 constexpr int THREADS = 320;
 constexpr int NCOMP = 256;
-constexpr int RING = 7;
+constexpr int RING = 4;
 constexpr int WST = 128 * 128;            // one 128-row x 64-column bf16 weight tile
 constexpr int NOPK = 8;                   // operand K blocks (64 tokens x 64 bf16 each, 128B swizzle)
 constexpr int OPB = NOPK * 8192;
-constexpr int NSTG = 5;                   // fp32 staging slots, 64 rows x 32 columns, 128B swizzle
+constexpr int NSTG = 11;                  // fp32 staging slots, 64 rows x 32 columns, 128B swizzle
 constexpr int STG = 8192;
 constexpr int TBL = 4096;                 // per-unit slice of the AdaRMS scale / GELU bias tables
 constexpr int REGION = OPB + NSTG * STG + TBL;  // operands + staging + table | attention | epilogue tile
@@ -333,25 +333,32 @@ __device__ void qkv_finalise(const PersistParams &p, int lv, size_t kl, int c, i
 
 // ---------------------------------------------------------------------------------------
 // attention unit: head h, key split s; 8 warps = 4 query blocks of 16 x 2 halves of head_dim.
-// Q_h rows and K/V rows arrive by 1-D bulk copies (prefix rows from the cache, suffix rows
-// from the finalised K_s / V_s).
+// Keys are taken in chunks of 32 that never mix prefix and suffix: chunks [0, npre) cover the
+// valid prefix (from the cache), chunks [npre, npre + nsuf) the C suffix keys (finalised
+// K_s / V_s).  Q_h and each K / V chunk arrive by TMA as four 64-column boxes with 128-byte
+// swizzle (element (r, c) of a [4][R][64] tile at block c/64, row r, 16-byte chunk
+// ((c%64)/8) ^ (r%8)).
 
 struct AttnCtx {
-  int lv, total, kps, nsplit, cap;
-  const bf16 *kv_k, *kv_v;  // prefix cache of this call (read once from the argument block)
+  int lv, npre, nsuf, cps, nsplit;
 };
 
+__device__ __forceinline__ uint32_t swz_addr(uint32_t base, int rows, int r, int c) {
+  return base + (c >> 6) * (rows * 128) + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+
 __device__ void attn_unit(const PersistParams &p, const Smem &sm, const AttnCtx &ac, int h, int s, int l,
-                          uint32_t &natt, int tid, unsigned epoch) {
-  bf16 *Qs = reinterpret_cast<bf16 *>(sm.op);
-  bf16 *Ks = Qs + 64 * LDS;
-  bf16 *Vs = Ks + KC * LDS;
+                          const CUtensorMap *tm_q, const CUtensorMap *tm_kc, const CUtensorMap *tm_vc,
+                          const CUtensorMap *tm_ks, const CUtensorMap *tm_vs, uint32_t &natt, int tid,
+                          unsigned epoch) {
+  uint8_t *Qs = sm.op;               // [4][64][64] bf16, swizzled
+  uint8_t *Ks = sm.op + 32768;       // [4][32][64]
+  uint8_t *Vs = sm.op + 49152;       // [4][32][64]
+  const uint32_t qa_ = smem_u32(Qs), ka_ = smem_u32(Ks), va_ = smem_u32(Vs);
   const int warp = tid >> 5, lane = tid & 31;
-  const int lv = ac.lv;
-  const int k_begin = s * ac.kps, k_end = min(ac.total, k_begin + ac.kps);
-  const size_t lay = (size_t)l * ac.cap * HD;  // batch 1
-  const bf16 *kpre = ac.kv_k + lay;
-  const bf16 *vpre = ac.kv_v + lay;
+  const int nch = ac.npre + ac.nsuf;
+  const int ch0 = s * ac.cps, ch1 = min(nch, ch0 + ac.cps);
+  const int cap = p.ca_cap;
 
   float o[16][4];
 #pragma unroll
@@ -359,41 +366,38 @@ __device__ void attn_unit(const PersistParams &p, const Smem &sm, const AttnCtx 
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const int g = lane >> 2, t = lane & 3;
   const int qb = warp & 3, dh = warp >> 2;
-  const bf16 *Qw = Qs + qb * 16 * LDS;
 
-  bool first = true;
 #pragma unroll 1
-  for (int c0 = k_begin; c0 < k_end || first; c0 += KC) {
-    const int nv = max(0, min(KC, k_end - c0));
+  for (int ch = ch0; ch < ch1; ++ch) {
+    const bool pre = ch < ac.npre;
+    const int nv = pre ? min(KC, ac.lv - ch * KC) : min(KC, p.C - (ch - ac.npre) * KC);
     named_sync();  // the previous chunk has been consumed
-    if (tid < 32) {
-      const uint32_t bytes = (first ? 64u * 512u : 0u) + (uint32_t)nv * 1024u;
-      if (tid == 0) mbar_arrive_expect_tx(sm.att, bytes);
-      __syncwarp();
-      if (first) {
-        bulk_load(Qs + lane * LDS, p.qb + (size_t)lane * 2048 + h * HD, 512, sm.att);
-        bulk_load(Qs + (lane + 32) * LDS, p.qb + (size_t)(lane + 32) * 2048 + h * HD, 512, sm.att);
+    if (tid == 0) {
+      const uint64_t pol = policy_evict_last();
+      const bool first = ch == ch0;
+      mbar_arrive_expect_tx(sm.att, (first ? 32768u : 0u) + 32768u);
+      if (first)
+        for (int b = 0; b < 4; ++b) tma_load_2d(Qs + b * 8192, tm_q, sm.att, h * HD + b * 64, 0, pol);
+      const CUtensorMap *mk = pre ? tm_kc : tm_ks;
+      const CUtensorMap *mv = pre ? tm_vc : tm_vs;
+      const int y = pre ? l * cap + ch * KC : (ch - ac.npre) * KC;
+      for (int b = 0; b < 4; ++b) {
+        tma_load_2d(Ks + b * 4096, mk, sm.att, b * 64, y, pol);
+        tma_load_2d(Vs + b * 4096, mv, sm.att, b * 64, y, pol);
       }
-      if (lane < nv) {
-        const int j = c0 + lane;
-        const bf16 *ksrc = j < lv ? kpre + (size_t)j * HD : p.ks + (size_t)(j - lv) * HD;
-        const bf16 *vsrc = j < lv ? vpre + (size_t)j * HD : p.vs + (size_t)(j - lv) * HD;
-        bulk_load(Ks + lane * LDS, ksrc, 512, sm.att);
-        bulk_load(Vs + lane * LDS, vsrc, 512, sm.att);
-      }
-    }
-    // key rows past the split's end are zero
-    for (int i = tid; i < (KC - nv) * 32; i += NCOMP) {
-      const int r = nv + i / 32, c8 = i % 32;
-      *reinterpret_cast<uint4 *>(Ks + r * LDS + c8 * 8) = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4 *>(Vs + r * LDS + c8 * 8) = make_uint4(0, 0, 0, 0);
     }
     wait_bar(sm.att, natt & 1, p.ctl, 651);
     ++natt;
+    // rows past the chunk's valid keys may hold anything: zero them (V is multiplied by p = 0)
+    for (int i = tid; i < (KC - nv) * 32; i += NCOMP) {
+      const int r = nv + (i >> 5), q16 = i & 31;  // 32 x 16 bytes per row (4 blocks x 8 chunks)
+      const int b = q16 >> 3, c16 = q16 & 7;
+      *reinterpret_cast<uint4 *>(Ks + b * 4096 + r * 128 + (c16 << 4)) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4 *>(Vs + b * 4096 + r * 128 + (c16 << 4)) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_shared();  // these generic writes precede the next chunk's TMA writes
     named_sync();
-    if (first && tid == 0) stamp(p, epoch, 4);
-    first = false;
-    if (nv == 0) break;
+    if (ch == ch0 && tid == 0) stamp(p, epoch, 4);
 
     float sc[4][4];
 #pragma unroll
@@ -401,13 +405,13 @@ __device__ void attn_unit(const PersistParams &p, const Smem &sm, const AttnCtx 
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(a0, a1, a2, a3, smem_u32(Qw + (lane & 15) * LDS + kk * 16 + (lane >> 4) * 8));
+      ldsm_x4(a0, a1, a2, a3, swz_addr(qa_, 64, qb * 16 + (lane & 15), kk * 16 + (lane >> 4) * 8));
 #pragma unroll
       for (int nt = 0; nt < 4; nt += 2) {
         uint32_t b0, b1, b2, b3;
         const int r = nt * 8 + (lane & 7) + ((lane >> 4) << 3);
         const int c = kk * 16 + ((lane >> 3) & 1) * 8;
-        ldsm_x4(b0, b1, b2, b3, smem_u32(Ks + r * LDS + c));
+        ldsm_x4(b0, b1, b2, b3, swz_addr(ka_, 32, r, c));
         mma_16816(sc[nt], a0, a1, a2, a3, b0, b1);
         mma_16816(sc[nt + 1], a0, a1, a2, a3, b2, b3);
       }
@@ -417,8 +421,8 @@ __device__ void attn_unit(const PersistParams &p, const Smem &sm, const AttnCtx 
     for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int key = c0 + nt * 8 + 2 * t + (e & 1);
-        const float v = (key < k_end) ? sc[nt][e] * p.scale_log2 : -INFINITY;
+        const int key = nt * 8 + 2 * t + (e & 1);
+        const float v = (key < nv) ? sc[nt][e] * p.scale_log2 : -INFINITY;
         sc[nt][e] = v;
         if (e < 2) cm0 = fmaxf(cm0, v); else cm1 = fmaxf(cm1, v);
       }
@@ -463,7 +467,7 @@ __device__ void attn_unit(const PersistParams &p, const Smem &sm, const AttnCtx 
         uint32_t b0, b1, b2, b3;
         const int r = kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
         const int c = dh * 128 + dt * 8 + (lane >> 4) * 8;
-        ldsm_x4_t(b0, b1, b2, b3, smem_u32(Vs + r * LDS + c));
+        ldsm_x4_t(b0, b1, b2, b3, swz_addr(va_, 32, r, c));
         mma_16816(o[dt], a0, a1, a2, a3, b0, b1);
         mma_16816(o[dt + 1], a0, a1, a2, a3, b2, b3);
       }
@@ -551,7 +555,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                  const __grid_constant__ CUtensorMap tm_rq, const __grid_constant__ CUtensorMap tm_rg,
                  const __grid_constant__ CUtensorMap tm_rh, const __grid_constant__ CUtensorMap tm_lh,
                  const __grid_constant__ CUtensorMap tm_lg, const __grid_constant__ CUtensorMap tm_lo,
-                 PersistParams p) {
+                 const __grid_constant__ CUtensorMap tm_lq, const __grid_constant__ CUtensorMap tm_kc,
+                 const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_ks,
+                 const __grid_constant__ CUtensorMap tm_vs, PersistParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem sm;
@@ -674,15 +680,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const CallArgs *ca = p.ca;
     AttnCtx ac;
     ac.lv = ca->valid_len[0];
-    if (ac.lv < 0 || ac.lv > ca->cap) {
+    if (ac.lv < 0 || ac.lv > p.ca_cap) {
       if (tid == 0 && c == 0) set_error(ctl, DEVERR_BOUNDS, 631);
-      ac.lv = ac.lv < 0 ? 0 : ca->cap;
+      ac.lv = ac.lv < 0 ? 0 : p.ca_cap;
     }
-    ac.total = ac.lv + C;
-    ac.cap = ca->cap;
-    ac.kv_k = ca->kv_k;
-    ac.kv_v = ca->kv_v;
-    ac.kps = p.attn_kps;
+    ac.npre = (ac.lv + KC - 1) / KC;
+    ac.nsuf = (C + KC - 1) / KC;
+    ac.cps = p.attn_cps;
     ac.nsplit = p.attn_splits;
 
     // ---- init: x = noise, h = action_in(x); zero the accumulators and the unused rows
@@ -724,7 +728,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             qkv_finalise(p, ac.lv, kl, c, ncta, C, tid);
             grid_sync(p, p.bar, ctl, epoch, ncta, tid);
             zero_slice(p.acc_qkv, (size_t)M * 2560, c, ncta, tid);
-            for (int u = c; u < NH * ac.nsplit; u += ncta) attn_unit(p, sm, ac, u % NH, u / NH, l, natt, tid, epoch);
+            for (int u = c; u < NH * ac.nsplit; u += ncta)
+              attn_unit(p, sm, ac, u % NH, u / NH, l, &tm_lq, &tm_kc, &tm_vc, &tm_ks, &tm_vs, natt, tid, epoch);
             grid_sync(p, p.bar, ctl, epoch, ncta, tid);
             combine_rows(p, ac.nsplit, c, ncta, C, tid);
             if (c == 0)
@@ -894,14 +899,13 @@ bool persistent_fits(int sm_count) {
   return blocks >= 1 && sm_count >= 64;
 }
 
-void persistent_attn_plan(int keys, int sm_count, int *splits, int *kps) {
-  const int chunks = (keys + pk::KC - 1) / pk::KC;
+void persistent_attn_plan(int cap, int chunk, int sm_count, int *splits, int *cps) {
+  const int chunks = (cap + pk::KC - 1) / pk::KC + (chunk + pk::KC - 1) / pk::KC;
   int s = persistent_max_splits(sm_count);
   if (s > chunks) s = chunks;
   if (s < 1) s = 1;
-  const int cps = (chunks + s - 1) / s;
-  *kps = cps * pk::KC;
-  *splits = (chunks + cps - 1) / cps;
+  *cps = (chunks + s - 1) / s;
+  *splits = (chunks + *cps - 1) / *cps;
 }
 
 cudaError_t persistent_launch(const PersistMaps &m, const PersistParams &p, int grid, cudaStream_t st) {
@@ -910,7 +914,9 @@ cudaError_t persistent_launch(const PersistMaps &m, const PersistParams &p, int 
                   const_cast<CUtensorMap *>(&m.r_qkv), const_cast<CUtensorMap *>(&m.r_gu),
                   const_cast<CUtensorMap *>(&m.r_h),   const_cast<CUtensorMap *>(&m.l_h),
                   const_cast<CUtensorMap *>(&m.l_gu),  const_cast<CUtensorMap *>(&m.l_o),
-                  const_cast<PersistParams *>(&p)};
+                  const_cast<CUtensorMap *>(&m.l_q),   const_cast<CUtensorMap *>(&m.l_kc),
+                  const_cast<CUtensorMap *>(&m.l_vc),  const_cast<CUtensorMap *>(&m.l_ks),
+                  const_cast<CUtensorMap *>(&m.l_vs),  const_cast<PersistParams *>(&p)};
   return cudaLaunchCooperativeKernel(reinterpret_cast<void *>(pk::k_persistent), dim3(grid), dim3(pk::THREADS), args,
                                      pk::SMEM, st);
 }

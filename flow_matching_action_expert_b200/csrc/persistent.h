@@ -15,7 +15,8 @@ struct PersistParams {
   int final_norm;
   float eps;
   float scale_log2;         // log2(e) / sqrt(head_dim)
-  int attn_splits, attn_kps;
+  int attn_splits, attn_cps;  // attention key splits and 32-key chunks per split
+  int ca_cap;                 // token stride of this call's prefix cache
   // folded weights and per-(step, layer) tables (library-owned)
   const bf16 *w_in;
   const float *b_in, *w_out, *b_out;
@@ -37,7 +38,7 @@ struct PersistParams {
 int persistent_smem_bytes();
 cudaError_t persistent_init_attributes();
 bool persistent_fits(int sm_count);
-void persistent_attn_plan(int keys, int sm_count, int *splits, int *kps);
+void persistent_attn_plan(int cap, int chunk, int sm_count, int *splits, int *cps);
 int persistent_max_splits(int sm_count);  // upper bound of the splits any plan returns
 // Tensor maps of the persistent kernel.
 struct PersistMaps {
@@ -45,6 +46,9 @@ struct PersistMaps {
   CUtensorMap r_qkv, r_gu, r_h;       // fp32 bulk-reduce targets acc_qkv, acc_gu, h (128 x 64 boxes)
   CUtensorMap l_h, l_gu;              // fp32 loads of h and acc_gu, 32-column x 64-row boxes, 128B swizzle
   CUtensorMap l_o;                    // bf16 load of the attention output, 64 x 64 boxes, 128B swizzle
+  CUtensorMap l_q;                    // bf16 finalised Q [64][2048], 64 x 64 boxes
+  CUtensorMap l_kc, l_vc;             // this call's prefix cache [L * cap][256], 64 x 32 boxes (per call)
+  CUtensorMap l_ks, l_vs;             // finalised suffix K / V [64][256], 64 x 32 boxes
 };
 cudaError_t persistent_launch(const PersistMaps &m, const PersistParams &p, int grid, cudaStream_t st);
 

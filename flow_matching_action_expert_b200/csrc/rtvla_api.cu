@@ -69,6 +69,8 @@ struct rtvla_ctx {
   CallArgs *args_dn = nullptr, *args_pf = nullptr, *args_tr = nullptr;
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_pwqkv, tm_pwo, tm_pwgu, tm_pwd;
   PersistMaps pmaps;                // tensor maps of the persistent engine
+  CUtensorMap tm_q64;               // finalised Q, 64-row boxes
+  const void *pk_cache_k = nullptr, *pk_cache_v = nullptr;  // prefix cache of the current call
   XMaps tm_op, tm_o, tm_mb, tm_pop, tm_po, tm_pmb;
   std::map<std::pair<int, int>, GraphEntry> graphs_dn, graphs_pf;
   std::map<int, int> kernels_per_call;
@@ -329,7 +331,10 @@ bool use_persistent(const rtvla_ctx *c, int batch) {
   return c->pers_ok && batch == 1;
 }
 
-cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, int cap, cudaStream_t st) {
+cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, const rtvla_kv *kv, cudaStream_t st) {
+  const int cap = kv->prefix_cap;
+  c->pk_cache_k = kv->k;
+  c->pk_cache_v = kv->v;
   PersistParams p;
   std::memset(&p, 0, sizeof(p));
   p.ca = dargs;
@@ -341,7 +346,12 @@ cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, int cap, cudaStream
   p.final_norm = c->cfg.final_norm;
   p.eps = c->cfg.rms_eps;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
-  persistent_attn_plan(cap + c->C, c->sm_count, &p.attn_splits, &p.attn_kps);
+  persistent_attn_plan(cap, c->C, c->sm_count, &p.attn_splits, &p.attn_cps);
+  p.ca_cap = cap;
+  // this call's prefix cache (batch 1): [L * cap][256] bf16, 32-key x 64-column boxes
+  if (!make_map(&c->pmaps.l_kc, c->pk_cache_k, (uint64_t)c->L * cap, HD, 32) ||
+      !make_map(&c->pmaps.l_vc, c->pk_cache_v, (uint64_t)c->L * cap, HD, 32))
+    return cudaErrorInvalidValue;
   p.w_in = c->w_in;
   p.b_in = c->b_in;
   p.w_out = c->w_out;
@@ -641,7 +651,8 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
             make_map(&c->tm_wo, c->w_o, (uint64_t)L * D, NQH * HD, 128) &&
             make_map(&c->tm_wgu, c->w_gu, (uint64_t)L * 2 * F, D, 128) &&
             make_map(&c->tm_wd, c->w_d, (uint64_t)L * D, F, 128) && make_xmaps(&c->tm_op, c->op, M, D) &&
-            make_xmaps(&c->tm_o, c->o, M, NQH * HD) && make_xmaps(&c->tm_mb, c->mb, M, F);
+            make_xmaps(&c->tm_o, c->o, M, NQH * HD) && make_xmaps(&c->tm_mb, c->mb, M, F) &&
+            make_map(&c->tm_q64, c->q, M, NQH * HD, 64);
   if (c->cfg.has_prefill) {
     ok = ok && make_map(&c->tm_pwqkv, c->pw_qkv, (uint64_t)L * 2560, DP, 128) &&
          make_map(&c->tm_pwo, c->pw_o, (uint64_t)L * DP, NQH * HD, 128) &&
@@ -668,9 +679,11 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
     pm.w_gu = c->tm_wgu;
     pm.w_d = c->tm_wd;
     pm.l_o = c->tm_o.m[0];
+    pm.l_q = c->tm_q64;
     if (!make_map_f32(&pm.r_qkv, c->acc_qkv, 64, 2560, 128, false) ||
         !make_map_f32(&pm.r_gu, c->acc_gu, 64, 2 * F, 128, false) || !make_map_f32(&pm.r_h, c->h, 64, D, 128, false) ||
-        !make_map_f32(&pm.l_h, c->h, 64, D, 32, true) || !make_map_f32(&pm.l_gu, c->acc_gu, 64, 2 * F, 32, true))
+        !make_map_f32(&pm.l_h, c->h, 64, D, 32, true) || !make_map_f32(&pm.l_gu, c->acc_gu, 64, 2 * F, 32, true) ||
+        !make_map(&pm.l_ks, c->ks, 256, HD, 32) || !make_map(&pm.l_vs, c->vs, 256, HD, 32))
       return RTVLA_ERR_CUDA;
     if (std::getenv("RTVLA_PHASE_STAMPS")) {
       c->pk_max_phases = c->S * (7 * c->L + 1) + 2;
@@ -799,7 +812,7 @@ rtvla_status rtvla_sample_actions(rtvla_ctx *c, const float *noise, const rtvla_
   if (c->engine == RTVLA_ENGINE_PERSISTENT && !use_persistent(c, kv->batch)) return RTVLA_ERR_UNSUPPORTED;
   if (use_persistent(c, kv->batch)) {
     if (cudaMemcpyAsync(c->args_dn, &a, sizeof(a), cudaMemcpyHostToDevice, st) != cudaSuccess) return RTVLA_ERR_CUDA;
-    if (launch_persistent(c, c->args_dn, kv->prefix_cap, st) != cudaSuccess) {
+    if (launch_persistent(c, c->args_dn, kv, st) != cudaSuccess) {
       cudaGetLastError();
       return RTVLA_ERR_CUDA;
     }
