@@ -40,7 +40,6 @@ def parse():
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--engine", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--no-flush", action="store_true")
     return p.parse_args()
 
 
@@ -123,6 +122,42 @@ class Clocks:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
+KERNEL_SOURCES = ("csrc/persistent.cu", "csrc/persistent.h", "csrc/common.cuh", "csrc/rtvla_api.cu")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "flow_matching_action_expert_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload_name, engine):
+    """DRAM bytes (read + write) per launch of the persistent kernel, from the committed ncu
+    summary of this workload.  None unless the summary's source hash equals the hash of the
+    sources now, i.e. the kernel has not changed since the counters were taken."""
+    if engine != "persistent":
+        return None
+    import re
+    slug = re.sub(r"[^0-9A-Za-z]+", "_", workload_name)
+    path = os.path.join(ROOT, "profiles", f"k_persistent_{slug}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if line.startswith("- ") and ": " in line:
+            k, v = line[2:].split(": ", 1)
+            fields[k.strip().strip("`")] = v.strip().strip("`")
+    if fields.get("source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -202,7 +237,7 @@ def run_ours(args, rank, world, local_rank):
     out = torch.empty_like(noise)
     kv = R.make_kv(k, v, vl, wl.batch, wl.prefix_cap)
     stream = torch.cuda.current_stream(dev)
-    flush = None if args.no_flush else torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
     def call():
         R.rtvla_sample_actions(ctx, noise, kv, out, stream)
@@ -221,8 +256,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     with Clocks(local_rank) as clk:
         for i in range(args.steps):
-            if flush is not None:
-                flush.fill_(float(i))          # L2 flush (256 MiB write) outside the timed events
+            flush.fill_(float(i))              # L2 flush (256 MiB write) outside the timed events
             starts[i].record(stream)
             call()
             ends[i].record(stream)
@@ -275,7 +309,7 @@ def run_ours(args, rank, world, local_rank):
     t_mem = bytes_loop / (hbm * 1e9)
     t_tc = flops_loop / (bf16_sus * 1e12)
     bound = "hbm" if t_mem >= t_tc else "tensor"
-    engine = {0: "auto", 1: "layered", 2: "persistent"}[args.engine]
+    engine = "persistent" if kernels == 1 else "layered"   # the engine the call actually ran
     line = {
         "metric": METRIC, "value": round(ms, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": False,
@@ -284,18 +318,19 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": wl.name, "batch": wl.batch, "chunk": wl.chunk, "prefix": wl.prefix_cap,
                    "valid_prefix": list(wl.valid_lens)[:4], "layers": wl.expert.n_layers,
                    "steps_per_loop": wl.expert.n_steps, "engine": engine, "parallelism": f"replicas{world}",
-                   "l2": ("flushed by a 256 MiB write between timed loops; weights (623 MB) exceed L2"
-                          if flush is not None else "not flushed; weights (623 MB) exceed L2")},
+                   "l2": "flushed by a 256 MiB write between timed loops; weights (623 MB) exceed L2"},
         "hbm_gbs_achieved": round(achieved_gbs, 1),
         "chunks_per_s": round(world * wl.batch / (ms * 1e-3), 2),
         "latency_ms": {"p10": round(float(np.percentile(per, 10)), 4), "p50": round(float(np.median(per)), 4),
                        "p90": round(float(np.percentile(per, 90)), 4)},
-        "roofline": {"bound": bound, "kernel": f"rtvla_sample_actions ({engine} engine, one call)",
+        "roofline": {"bound": bound,
+                     "kernel": ("k_persistent (one launch = one call)" if engine == "persistent"
+                                else "rtvla_sample_actions (layered engine, one graph replay)"),
                      "achieved": round(achieved_gbs if bound == "hbm" else achieved_tf, 1),
                      "peak": hbm if bound == "hbm" else bf16_sus,
                      "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
                      "frac": round((achieved_gbs / hbm) if bound == "hbm" else (achieved_tf / bf16_sus), 4),
-                     "traffic": None, "peak_source": src,
+                     "traffic": measured_traffic(wl.name, engine), "peak_source": src,
                      "algorithmic_bytes_per_launch": int(bytes_loop), "algorithmic_flops_per_launch": int(flops_loop),
                      "roofline_ms": round(max(t_mem, t_tc) * 1e3, 4)},
         "e2e": {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
