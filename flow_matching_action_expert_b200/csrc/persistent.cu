@@ -29,19 +29,20 @@ namespace pk {
 
 constexpr int THREADS = 320;
 constexpr int NCOMP = 256;
-constexpr int RING = 4;
+constexpr int RING = 5;
 constexpr int WST = 128 * 128;            // one 128-row x 64-column bf16 weight tile
 constexpr int NOPK = 8;                   // operand K blocks (64 tokens x 64 bf16 each, 128B swizzle)
 constexpr int OPB = NOPK * 8192;
-constexpr int NSTG = 11;                  // fp32 staging slots, 64 rows x 32 columns, 128B swizzle
-constexpr int STG = 8192;
+constexpr int NGRP = 2;                   // fp32 staging groups (double buffer)
+constexpr int STG = 8192;                 // one staged tile: 64 rows x 32 columns, 128B swizzle
+constexpr int GRPB = 4 * STG;             // a group: 4 tiles, filled by one or two 3-D TMA boxes
 constexpr int TBL = 4096;                 // per-unit slice of the AdaRMS scale / GELU bias tables
-constexpr int REGION = OPB + NSTG * STG + TBL;  // operands + staging + table | attention | epilogue tile
+constexpr int REGION = OPB + NGRP * GRPB + TBL;  // operands + staging + table | attention | epilogue tile
 constexpr int LDS = 264;                  // attention shared rows (bf16), 528 bytes
 constexpr int KC = 32;                    // attention keys per chunk
 constexpr int ATT_BYTES = (64 + 2 * KC) * LDS * 2;
 static_assert(ATT_BYTES <= REGION, "attention tiles must fit the shared region");
-constexpr int NBARS = 2 * RING + NOPK + NSTG + 4;
+constexpr int NBARS = 2 * RING + NOPK + NGRP + 4;
 constexpr int SMEM = RING * WST + REGION + 1024 + NBARS * 8 + 64;
 constexpr int D = 1024, F = 4096, HD = 256, NH = 8, A = 32;
 constexpr int MAXSPLIT = 18;
@@ -184,21 +185,43 @@ __device__ __forceinline__ uint4 *op_chunk(uint8_t *op, int j, int r, int cc) {
   return reinterpret_cast<uint4 *>(op + j * 8192 + r * 128 + ((cc ^ (r & 7)) << 4));
 }
 
-// Builds the bf16 operand of one GEMM unit from fp32 tiles staged by TMA, one 32-column piece
-// at a time, and releases each 64-wide K block to the MMA as soon as it is complete.
+// Builds the bf16 operand of one GEMM unit from fp32 tiles staged by TMA and releases each
+// 64-wide K block to the MMA as soon as it is complete.  Staging runs in groups of four
+// 64-row x 32-column tiles, double-buffered: QKV / GU fetch a group as one 3-D box of four
+// consecutive column tiles of h; DN as two boxes (two gate tiles, the two matching up tiles).
+// One wait, one proxy fence and one barrier per group; the group after next is issued as soon
+// as a buffer is consumed.
 //   QKV / GU:  bf16(h * (1 + scale)); designated units add the slice's sum of squares of h
 //   DN:        bf16(GELU_tanh(r*g + bg) * (r*u + bu)) from the gate/up accumulator
 __device__ void build_operand(const PersistParams &p, const Smem &sm, const CUtensorMap *tm_lh,
                               const CUtensorMap *tm_lg, int kind, int kb0, int nkb, const float *s1p,
                               const float *bias, float *ss, bool stats, int M, uint32_t &g, uint32_t &ntbl,
                               int tid) {
-  const int cpp = kind == DN ? 2 : 1;  // staged tiles per piece
-  const int npieces = 2 * nkb;
-  const int nch = npieces * cpp;
+  const bool dn = kind == DN;
+  const int npieces = 2 * nkb;          // 32-column pieces of the unit's K slice
+  const int ppg = dn ? 2 : 4;           // pieces per group
+  const int ngroups = (npieces + ppg - 1) / ppg;
   const uint32_t g0 = g;
-  const int ncol = nkb * 64;           // table slice: scale (QKV, GU) or gate | up bias (DN)
+  const int ncol = nkb * 64;            // table slice: scale (QKV, GU) or gate | up bias (DN)
+  uint64_t pol = 0;
+  // group q covers pieces [q * ppg, q * ppg + ppg) (a short last group reads its box's spare
+  // tiles from the neighbouring columns, or zero fill past the end; they are never used)
+  auto issue = [&](int q) {
+    const int buf = (g0 + q) % NGRP;
+    uint8_t *dst = sm.stg + buf * GRPB;
+    const int z = (kb0 * 64) / 32 + q * ppg;
+    mbar_arrive_expect_tx(&sm.stgb[buf], GRPB);
+    if (dn) {
+      tma_load_3d(dst, tm_lg, &sm.stgb[buf], 0, 0, z, pol);
+      tma_load_3d(dst + 2 * STG, tm_lg, &sm.stgb[buf], 0, 0, z + F / 32, pol);
+    } else {
+      tma_load_3d(dst, tm_lh, &sm.stgb[buf], 0, 0, z, pol);
+    }
+  };
   if (tid == 0) {
-    if (kind == DN) {
+    pol = policy_evict_last();
+    for (int q = 0; q < ngroups && q < NGRP; ++q) issue(q);
+    if (dn) {
       mbar_arrive_expect_tx(sm.tblb, 2 * ncol * 4);
       bulk_load(sm.tbl, bias + kb0 * 64, ncol * 4, sm.tblb);
       bulk_load(sm.tbl + ncol, bias + F + kb0 * 64, ncol * 4, sm.tblb);
@@ -206,82 +229,62 @@ __device__ void build_operand(const PersistParams &p, const Smem &sm, const CUte
       mbar_arrive_expect_tx(sm.tblb, ncol * 4);
       bulk_load(sm.tbl, s1p + kb0 * 64, ncol * 4, sm.tblb);
     }
-    const uint64_t pol = policy_evict_last();
-    for (int ci = 0; ci < nch && ci < NSTG; ++ci) {
-      const int slot = (g0 + ci) % NSTG;
-      const int col = kb0 * 64 + (ci / cpp) * 32;
-      mbar_arrive_expect_tx(&sm.stgb[slot], STG);
-      if (kind == DN)
-        tma_load_2d(sm.stg + slot * STG, tm_lg, &sm.stgb[slot], (ci & 1) ? F + col : col, 0, pol);
-      else
-        tma_load_2d(sm.stg + slot * STG, tm_lh, &sm.stgb[slot], col, 0, pol);
-    }
   }
   const int r = tid >> 2, sub = tid & 3;
   float acc = 0.f;
   float rr = 0.f;
-  if (kind == DN && r < M) rr = rsqrtf(__ldcg(ss + r) * (1.0f / D) + p.eps);
+  if (dn && r < M) rr = rsqrtf(__ldcg(ss + r) * (1.0f / D) + p.eps);
   wait_bar(sm.tblb, ntbl & 1, p.ctl, 642);
   ++ntbl;
-  for (int pc = 0; pc < npieces; ++pc) {
-    const int col = pc * 32 + sub * 8;  // column within the unit's K slice
-    const int j = pc >> 1, cc = (pc & 1) * 4 + sub;
-    for (int t = 0; t < cpp; ++t) {
-      const uint32_t gi = g0 + pc * cpp + t;
-      wait_bar(&sm.stgb[gi % NSTG], (gi / NSTG) & 1, p.ctl, 641);
-    }
-    uint4 out = make_uint4(0, 0, 0, 0);
-    if (r < M) {
-      float v[8];
-      if (kind == DN) {
-        float u[8];
-        stg_read8(sm.stg + ((g0 + pc * 2) % NSTG) * STG, r, 2 * sub, v);
-        stg_read8(sm.stg + ((g0 + pc * 2 + 1) % NSTG) * STG, r, 2 * sub, u);
-        const float4 bg0 = *reinterpret_cast<const float4 *>(sm.tbl + col);
-        const float4 bg1 = *reinterpret_cast<const float4 *>(sm.tbl + col + 4);
-        const float4 bu0 = *reinterpret_cast<const float4 *>(sm.tbl + ncol + col);
-        const float4 bu1 = *reinterpret_cast<const float4 *>(sm.tbl + ncol + col + 4);
-        const float bgv[8] = {bg0.x, bg0.y, bg0.z, bg0.w, bg1.x, bg1.y, bg1.z, bg1.w};
-        const float buv[8] = {bu0.x, bu0.y, bu0.z, bu0.w, bu1.x, bu1.y, bu1.z, bu1.w};
+  for (int q = 0; q < ngroups; ++q) {
+    const uint32_t gq = g0 + q;
+    const uint8_t *grp = sm.stg + (gq % NGRP) * GRPB;
+    wait_bar(&sm.stgb[gq % NGRP], (gq / NGRP) & 1, p.ctl, 641);
+    const int p0 = q * ppg, pe = p0 + ppg < npieces ? p0 + ppg : npieces;
+    for (int pc = p0; pc < pe; ++pc) {
+      const int col = pc * 32 + sub * 8;  // column within the unit's K slice
+      const int j = pc >> 1, cc = (pc & 1) * 4 + sub;
+      uint4 out = make_uint4(0, 0, 0, 0);
+      if (r < M) {
+        float v[8];
+        if (dn) {
+          float u[8];
+          stg_read8(grp + (pc - p0) * STG, r, 2 * sub, v);
+          stg_read8(grp + (2 + pc - p0) * STG, r, 2 * sub, u);
+          const float4 bg0 = *reinterpret_cast<const float4 *>(sm.tbl + col);
+          const float4 bg1 = *reinterpret_cast<const float4 *>(sm.tbl + col + 4);
+          const float4 bu0 = *reinterpret_cast<const float4 *>(sm.tbl + ncol + col);
+          const float4 bu1 = *reinterpret_cast<const float4 *>(sm.tbl + ncol + col + 4);
+          const float bgv[8] = {bg0.x, bg0.y, bg0.z, bg0.w, bg1.x, bg1.y, bg1.z, bg1.w};
+          const float buv[8] = {bu0.x, bu0.y, bu0.z, bu0.w, bu1.x, bu1.y, bu1.z, bu1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = gelu_tanh_fast(rr * v[e] + bgv[e]) * (rr * u[e] + buv[e]);
-      } else {
-        stg_read8(sm.stg + ((g0 + pc) % NSTG) * STG, r, 2 * sub, v);
-        const float4 s0 = *reinterpret_cast<const float4 *>(sm.tbl + col);
-        const float4 s1 = *reinterpret_cast<const float4 *>(sm.tbl + col + 4);
-        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+          for (int e = 0; e < 8; ++e) v[e] = gelu_tanh_fast(rr * v[e] + bgv[e]) * (rr * u[e] + buv[e]);
+        } else {
+          stg_read8(grp + (pc - p0) * STG, r, 2 * sub, v);
+          const float4 s0 = *reinterpret_cast<const float4 *>(sm.tbl + col);
+          const float4 s1 = *reinterpret_cast<const float4 *>(sm.tbl + col + 4);
+          const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          acc += v[e] * v[e];
-          v[e] *= sv[e];
+          for (int e = 0; e < 8; ++e) {
+            acc += v[e] * v[e];
+            v[e] *= sv[e];
+          }
         }
+        out.x = pack_bf16(v[0], v[1]);
+        out.y = pack_bf16(v[2], v[3]);
+        out.z = pack_bf16(v[4], v[5]);
+        out.w = pack_bf16(v[6], v[7]);
       }
-      out.x = pack_bf16(v[0], v[1]);
-      out.y = pack_bf16(v[2], v[3]);
-      out.z = pack_bf16(v[4], v[5]);
-      out.w = pack_bf16(v[6], v[7]);
+      *op_chunk(sm.op, j, r, cc) = out;
     }
-    *op_chunk(sm.op, j, r, cc) = out;
-    if (pc & 1) fence_proxy_async_shared();  // K block j complete: make it visible to the MMA
+    fence_proxy_async_shared();  // the group's K blocks are complete: visible to the MMA
     named_sync();
     if (tid == 0) {
-      if (pc & 1) mbar_arrive(&sm.opf[j]);
-      const uint64_t pol = policy_evict_last();
-      for (int t = 0; t < cpp; ++t) {
-        const int ci = pc * cpp + t + NSTG;  // the tile that reuses the slot just consumed
-        if (ci < nch) {
-          const int slot = (g0 + ci) % NSTG;
-          const int ccol = kb0 * 64 + (ci / cpp) * 32;
-          mbar_arrive_expect_tx(&sm.stgb[slot], STG);
-          if (kind == DN)
-            tma_load_2d(sm.stg + slot * STG, tm_lg, &sm.stgb[slot], (ci & 1) ? F + ccol : ccol, 0, pol);
-          else
-            tma_load_2d(sm.stg + slot * STG, tm_lh, &sm.stgb[slot], ccol, 0, pol);
-        }
-      }
+      for (int j = p0 >> 1; j < (pe >> 1); ++j) mbar_arrive(&sm.opf[j]);
+      if (q + NGRP < ngroups) issue(q + NGRP);  // refill the buffer just consumed
     }
   }
-  g = g0 + nch;
+  g = g0 + ngroups;
   if (stats) {
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
@@ -547,6 +550,31 @@ __device__ void combine_rows(const PersistParams &p, int nsplit, int c, int ncta
   }
 }
 
+// L2 prefetch of the table slices this CTA's units of GEMM phase gp will read: the operand
+// scale or GELU bias slice, and the residual gate of the epilogue.  The weight producer issues
+// it one phase ahead, so these small per-(step, layer) reads do not wait on HBM.
+__device__ void prefetch_tables(const PersistParams &p, int gp, int c, int ncta) {
+  if (gp >= p.S * p.L * 4) return;
+  const int kind = gp & 3;
+  const size_t kl = (size_t)(gp >> 2);
+  for (int u = first_unit(gp, c, ncta); u < units(kind); u += ncta) {
+    int nt, kb0, kb1;
+    unit_kb(kind, u, nt, kb0, kb1);
+    const uint32_t bytes = (uint32_t)(kb1 - kb0) * 64 * 4;
+    if (kind == QKV) {
+      bulk_prefetch_l2(p.s1p_attn + kl * D + kb0 * 64, bytes);
+    } else if (kind == GU) {
+      bulk_prefetch_l2(p.s1p_ffn + kl * D + kb0 * 64, bytes);
+    } else if (kind == DN) {
+      bulk_prefetch_l2(p.bias_gu + kl * 2 * F + kb0 * 64, bytes);
+      bulk_prefetch_l2(p.bias_gu + kl * 2 * F + F + kb0 * 64, bytes);
+      bulk_prefetch_l2(p.gate_ffn + kl * D + nt * 128, 512);
+    } else {
+      bulk_prefetch_l2(p.gate_attn + kl * D + nt * 128, 512);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -564,13 +592,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   sm.ring = smem;
   sm.op = smem + RING * WST;
   sm.stg = sm.op + OPB;
-  sm.tbl = reinterpret_cast<float *>(sm.stg + NSTG * STG);
+  sm.tbl = reinterpret_cast<float *>(sm.stg + NGRP * GRPB);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm.op + REGION);
   sm.full = bars;
   sm.empty = bars + RING;
   sm.opf = bars + 2 * RING;
   sm.stgb = sm.opf + NOPK;
-  sm.acc_ready = sm.stgb + NSTG;
+  sm.acc_ready = sm.stgb + NGRP;
   sm.drain = sm.acc_ready + 1;
   sm.att = sm.drain + 1;
   sm.tblb = sm.att + 1;
@@ -608,6 +636,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int l = 0; l < L && ok; ++l)
           for (int kind = 0; kind < 4 && ok; ++kind) {
             const int gp = (k * L + l) * 4 + kind;
+            prefetch_tables(p, gp + 1, c, ncta);
             for (int u = first_unit(gp, c, ncta); u < units(kind) && ok; u += ncta) {
               int nt, kb0, kb1;
               unit_kb(kind, u, nt, kb0, kb1);

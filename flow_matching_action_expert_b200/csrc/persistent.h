@@ -44,7 +44,8 @@ int persistent_max_splits(int sm_count);  // upper bound of the splits any plan 
 struct PersistMaps {
   CUtensorMap w_qkv, w_o, w_gu, w_d;  // stacked bf16 weights, 64-column x 128-row boxes, 128B swizzle
   CUtensorMap r_qkv, r_gu, r_h;       // fp32 bulk-reduce targets acc_qkv, acc_gu, h (128 x 64 boxes)
-  CUtensorMap l_h, l_gu;              // fp32 loads of h and acc_gu, 32-column x 64-row boxes, 128B swizzle
+  CUtensorMap l_h, l_gu;              // fp32 loads of h (4 x 8 KB tiles per box) and acc_gu (2 per box):
+                                      // 3-D {32 cols, 64 rows, column blocks}, 128B swizzle per tile
   CUtensorMap l_o;                    // bf16 load of the attention output, 64 x 64 boxes, 128B swizzle
   CUtensorMap l_q;                    // bf16 finalised Q [64][2048], 64 x 64 boxes
   CUtensorMap l_kc, l_vc;             // this call's prefix cache [L * cap][256], 64 x 32 boxes (per call)

@@ -123,6 +123,20 @@ bool make_map_f32(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols
   return r == CUDA_SUCCESS;
 }
 
+// fp32 [64][cols] row-major, seen as 3-D {32 columns, 64 rows, cols / 32 column blocks} with
+// strides (row cols * 4 B, block 128 B): one box of `blocks` column blocks lands in shared
+// memory as that many consecutive 8 KB tiles [64 rows][32 columns], each with 128-byte swizzle.
+bool make_map_f32_blocks(CUtensorMap *m, const void *base, uint64_t cols, uint32_t blocks) {
+  cuuint64_t dims[3] = {32, 64, cols / 32};
+  cuuint64_t strides[2] = {cols * 4, 128};
+  cuuint32_t box[3] = {32, 64, blocks};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_xmaps(XMaps *x, const void *base, uint64_t rows, uint64_t cols) {
   return make_map(&x->m[0], base, rows, cols, 64) && make_map(&x->m[1], base, rows, cols, 128) &&
          make_map(&x->m[2], base, rows, cols, 256);
@@ -682,7 +696,7 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
     pm.l_q = c->tm_q64;
     if (!make_map_f32(&pm.r_qkv, c->acc_qkv, 64, 2560, 128, false) ||
         !make_map_f32(&pm.r_gu, c->acc_gu, 64, 2 * F, 128, false) || !make_map_f32(&pm.r_h, c->h, 64, D, 128, false) ||
-        !make_map_f32(&pm.l_h, c->h, 64, D, 32, true) || !make_map_f32(&pm.l_gu, c->acc_gu, 64, 2 * F, 32, true) ||
+        !make_map_f32_blocks(&pm.l_h, c->h, D, 4) || !make_map_f32_blocks(&pm.l_gu, c->acc_gu, 2 * F, 2) ||
         !make_map(&pm.l_ks, c->ks, 256, HD, 32) || !make_map(&pm.l_vs, c->vs, 256, HD, 32))
       return RTVLA_ERR_CUDA;
     if (std::getenv("RTVLA_PHASE_STAMPS")) {
