@@ -211,6 +211,13 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *m, const vo
                "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
+// 2-D bulk tensor store of a shared-memory box to global memory (bulk async-group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // the shared source of every committed bulk operation has been read
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

@@ -10,7 +10,9 @@
 // "res + (x @ W) * gate" of the Realtime-VLA tech blog, kernel list "matmul_small_res_gate").
 //
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer and TMEM owner, warps 2..5 =
-// epilogue (TMEM -> registers -> global).  Every wait is bounded (DevCtl::timeout_ns).
+// epilogue: TMEM -> registers (x gate) -> a [TN tokens][128 features] fp32 tile in the freed
+// pipeline stages -> one TMA bulk reduce-add (split K or accumulate) or bulk store per 64
+// tokens.  Every wait is bounded (DevCtl::timeout_ns).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,7 +30,8 @@ struct GemmCfg {
 
 template <int TN>
 __global__ void __launch_bounds__(192, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, GemmParams p) {
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+              const __grid_constant__ CUtensorMap tmO, GemmParams p) {
   using G = GemmCfg<TN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -95,29 +98,39 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(done);
     }
   } else if (nkb > 0) {
-    // epilogue: warp (2..5) & 3 selects the TMEM lane quadrant it may access
+    // epilogue: warp (2..5) & 3 selects the TMEM lane quadrant it may access; the tile reuses
+    // the pipeline stages (every TMA load into them has been consumed once `done` fires)
+    static_assert(TN * 128 * 4 <= G::STAGES * G::STAGE, "epilogue tile fits the stages");
+    float *tile = reinterpret_cast<float *>(smem);
     const int q = warp & 3;
+    const int nl = q * 32 + lane;
     if (mbar_wait(done, 0, p.ctl, 103)) {
       tc_fence_after();
-      const int n = n0 + q * 32 + lane;
-      const float sc = p.col_scale ? p.col_scale[n] : 1.0f;
+      const float sc = p.col_scale ? p.col_scale[n0 + nl] : 1.0f;
 #pragma unroll 1
       for (int c = 0; c < TN; c += 32) {
-        if (m0 + c >= p.M) break;
         float v[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+        if (m0 + c < p.M) {
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = m0 + c + j;
-          if (m < p.M) {
-            float *o = p.out + (size_t)m * p.ldo + n;
-            if (p.atomic)
-              atomicAdd(o, v[j] * sc);
-            else
-              *o = v[j] * sc;
-          }
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
         }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) tile[(c + j) * 128 + nl] = (m0 + c + j < p.M) ? v[j] * sc : 0.f;
       }
+    }
+    fence_proxy_async_shared();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 2 && lane == 0) {
+      for (int t = 0; t < TN && m0 + t < p.M; t += 64) {
+        if (p.atomic)
+          tma_reduce_add_2d(&tmO, tile + t * 128, n0, m0 + t);
+        else
+          tma_store_2d(&tmO, tile + t * 128, n0, m0 + t);
+      }
+      bulk_commit();
+      bulk_wait_read0();  // the tile must stay valid until the bulk copies have read it
     }
   }
   tc_fence_before();
@@ -130,11 +143,11 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 template <int TN>
-static cudaError_t launch_tn(const CUtensorMap &tmW, const CUtensorMap &tmX, const GemmParams &p, int n_tiles,
-                             int m_tiles, int splits, cudaStream_t st) {
+static cudaError_t launch_tn(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmO,
+                             const GemmParams &p, int n_tiles, int m_tiles, int splits, cudaStream_t st) {
   using G = GemmCfg<TN>;
   dim3 grid(n_tiles, m_tiles, splits);
-  k_gemm_tc<TN><<<grid, 192, G::SMEM, st>>>(tmW, tmX, p);
+  k_gemm_tc<TN><<<grid, 192, G::SMEM, st>>>(tmW, tmX, tmO, p);
   return cudaGetLastError();
 }
 
@@ -150,7 +163,9 @@ cudaError_t gemm_init_attributes() {
 // Chooses the token tile and the K split so that about one wave of 148 SMs is busy.
 GemmPlan gemm_plan(int M, int N, int K, int sm_count) {
   GemmPlan g;
-  g.tn = (M <= 64) ? 64 : (M <= 1024 ? 128 : 256);
+  // a 128 x 256 x 16 MMA costs about as much as 128 x 128 x 16 (and 128 x 64 x 16) on sm_100a,
+  // so past 128 rows the widest token tile wins even with its padding
+  g.tn = (M <= 64) ? 64 : (M <= 128 ? 128 : 256);
   g.m_tiles = (M + g.tn - 1) / g.tn;
   g.n_tiles = N / 128;
   const int kb_total = K / 64;
@@ -166,8 +181,8 @@ GemmPlan gemm_plan(int M, int N, int K, int sm_count) {
 int gemm_tile_index(int tn) { return tn <= 64 ? 0 : (tn <= 128 ? 1 : 2); }
 
 cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int M, int N, int K, float *out,
-                        int ldo, const float *col_scale, bool accumulate, DevCtl *ctl, int sm_count,
-                        cudaStream_t st) {
+                        const CUtensorMap &tmO, int ldo, const float *col_scale, bool accumulate, DevCtl *ctl,
+                        int sm_count, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   GemmPlan g = gemm_plan(M, N, K, sm_count);
   GemmParams p;
@@ -183,9 +198,9 @@ cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int
   p.ctl = ctl;
   const CUtensorMap &tmX = xm.m[gemm_tile_index(g.tn)];
   switch (g.tn) {
-    case 64: return launch_tn<64>(tmW, tmX, p, g.n_tiles, g.m_tiles, g.splits, st);
-    case 128: return launch_tn<128>(tmW, tmX, p, g.n_tiles, g.m_tiles, g.splits, st);
-    default: return launch_tn<256>(tmW, tmX, p, g.n_tiles, g.m_tiles, g.splits, st);
+    case 64: return launch_tn<64>(tmW, tmX, tmO, p, g.n_tiles, g.m_tiles, g.splits, st);
+    case 128: return launch_tn<128>(tmW, tmX, tmO, p, g.n_tiles, g.m_tiles, g.splits, st);
+    default: return launch_tn<256>(tmW, tmX, tmO, p, g.n_tiles, g.m_tiles, g.splits, st);
   }
 }
 

@@ -37,9 +37,10 @@ cudaError_t gemm_init_attributes();
 
 // out[m][n] (+)= col_scale[n] * sum_k X[m][k] W[w_row0 + n][k].  `accumulate` adds into the
 // existing contents of out; otherwise out must be zero when the plan splits K.
+// tmO: fp32 map of `out` ([rows][ldo], 128-column x 64-row boxes, no swizzle)
 cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int M, int N, int K, float *out,
-                        int ldo, const float *col_scale, bool accumulate, DevCtl *ctl, int sm_count,
-                        cudaStream_t st);
+                        const CUtensorMap &tmO, int ldo, const float *col_scale, bool accumulate, DevCtl *ctl,
+                        int sm_count, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------
 // attention (8 query heads share one KV head, head_dim 256)

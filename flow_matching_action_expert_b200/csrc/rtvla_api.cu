@@ -68,6 +68,8 @@ struct rtvla_ctx {
   DevCtl *ctl = nullptr;
   CallArgs *args_dn = nullptr, *args_pf = nullptr, *args_tr = nullptr;
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_pwqkv, tm_pwo, tm_pwgu, tm_pwd;
+  // fp32 GEMM outputs of the layered engine, 128-column x 64-row boxes (bulk store / reduce-add)
+  CUtensorMap tmo_qkv, tmo_h, tmo_gu, tmo_pqkv, tmo_px, tmo_pgu;
   PersistMaps pmaps;                // tensor maps of the persistent engine
   CUtensorMap tm_q64;               // finalised Q, 64-row boxes
   const void *pk_cache_k = nullptr, *pk_cache_v = nullptr;  // prefix cache of the current call
@@ -245,20 +247,20 @@ cudaError_t enqueue_denoise(rtvla_ctx *c, const CallArgs *dargs, int B, int cap,
     for (int l = 0; l < L; ++l) {
       const size_t kl = (size_t)k * L + l;
       CKN(launch_adanorm(c->h, c->s1p_attn + kl * D, c->op, c->r, M, eps, st));
-      CKN(gemm_launch(c->tm_wqkv, l * 2560, c->tm_op, M, 2560, D, c->acc_qkv, 2560, nullptr, false, c->ctl,
+      CKN(gemm_launch(c->tm_wqkv, l * 2560, c->tm_op, M, 2560, D, c->acc_qkv, c->tmo_qkv, 2560, nullptr, false, c->ctl,
                       c->sm_count, st));
       CKN(launch_qkv_post(c->acc_qkv, c->r, c->bias_qkv + kl * 2560, dargs, C, c->rope_cos, c->rope_sin,
                           c->rope_rows, c->q, c->ks, c->vs, M, c->ctl, st));
       ap.layer = l;
       CKN(attn_launch(ap, B, st));
       if (ap.n_splits > 1) ++n;
-      CKN(gemm_launch(c->tm_wo, l * D, c->tm_o, M, D, NQH * HD, c->h, D, c->gate_attn + kl * D, true, c->ctl,
+      CKN(gemm_launch(c->tm_wo, l * D, c->tm_o, M, D, NQH * HD, c->h, c->tmo_h, D, c->gate_attn + kl * D, true, c->ctl,
                       c->sm_count, st));
       CKN(launch_adanorm(c->h, c->s1p_ffn + kl * D, c->op, c->r, M, eps, st));
-      CKN(gemm_launch(c->tm_wgu, l * 2 * F, c->tm_op, M, 2 * F, D, c->acc_gu, 2 * F, nullptr, false, c->ctl,
+      CKN(gemm_launch(c->tm_wgu, l * 2 * F, c->tm_op, M, 2 * F, D, c->acc_gu, c->tmo_gu, 2 * F, nullptr, false, c->ctl,
                       c->sm_count, st));
       CKN(launch_gelu_mul(c->acc_gu, c->r, c->bias_gu + kl * 2 * F, c->mb, M, F, st));
-      CKN(gemm_launch(c->tm_wd, l * D, c->tm_mb, M, D, F, c->h, D, c->gate_ffn + kl * D, true, c->ctl,
+      CKN(gemm_launch(c->tm_wd, l * D, c->tm_mb, M, D, F, c->h, c->tmo_h, D, c->gate_ffn + kl * D, true, c->ctl,
                       c->sm_count, st));
       if (trace && k == last_step)
         CKR(cudaMemcpyAsync(trace + (size_t)(l + 1) * M * D, c->h, (size_t)M * D * 4, cudaMemcpyDeviceToDevice,
@@ -297,20 +299,20 @@ cudaError_t enqueue_prefill(rtvla_ctx *c, const CallArgs *dargs, int B, int P, c
   ap.ctl = c->ctl;
   for (int l = 0; l < L; ++l) {
     CKN(launch_rmsnorm(c->px, c->pop, M, DP, eps, st));
-    CKN(gemm_launch(c->tm_pwqkv, l * 2560, c->tm_pop, M, 2560, DP, c->pacc, 2560, nullptr, false, c->ctl,
+    CKN(gemm_launch(c->tm_pwqkv, l * 2560, c->tm_pop, M, 2560, DP, c->pacc, c->tmo_pqkv, 2560, nullptr, false, c->ctl,
                     c->sm_count, st));
     CKN(launch_pf_qkv_post(c->pacc, dargs, l, P, c->rope_cos, c->rope_sin, c->rope_rows, c->pq, M, c->ctl, st));
     if (l == L - 1) break;  // the last layer only provides K/V to the expert
     ap.layer = l;
     CKN(attn_launch(ap, B, st));
     if (ap.n_splits > 1) ++n;
-    CKN(gemm_launch(c->tm_pwo, l * DP, c->tm_po, M, DP, NQH * HD, c->px, DP, nullptr, true, c->ctl, c->sm_count,
-                    st));
+    CKN(gemm_launch(c->tm_pwo, l * DP, c->tm_po, M, DP, NQH * HD, c->px, c->tmo_px, DP, nullptr, true, c->ctl,
+                    c->sm_count, st));
     CKN(launch_rmsnorm(c->px, c->pop, M, DP, eps, st));
-    CKN(gemm_launch(c->tm_pwgu, l * 2 * FP, c->tm_pop, M, 2 * FP, DP, c->pacc, 2 * FP, nullptr, false, c->ctl,
+    CKN(gemm_launch(c->tm_pwgu, l * 2 * FP, c->tm_pop, M, 2 * FP, DP, c->pacc, c->tmo_pgu, 2 * FP, nullptr, false, c->ctl,
                     c->sm_count, st));
     CKN(launch_gelu_mul(c->pacc, nullptr, nullptr, c->pmb, M, FP, st));
-    CKN(gemm_launch(c->tm_pwd, l * DP, c->tm_pmb, M, DP, FP, c->px, DP, nullptr, true, c->ctl, c->sm_count, st));
+    CKN(gemm_launch(c->tm_pwd, l * DP, c->tm_pmb, M, DP, FP, c->px, c->tmo_px, DP, nullptr, true, c->ctl, c->sm_count, st));
   }
   *kernels = n;
   return cudaSuccess;
@@ -666,14 +668,16 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
             make_map(&c->tm_wgu, c->w_gu, (uint64_t)L * 2 * F, D, 128) &&
             make_map(&c->tm_wd, c->w_d, (uint64_t)L * D, F, 128) && make_xmaps(&c->tm_op, c->op, M, D) &&
             make_xmaps(&c->tm_o, c->o, M, NQH * HD) && make_xmaps(&c->tm_mb, c->mb, M, F) &&
-            make_map(&c->tm_q64, c->q, M, NQH * HD, 64);
+            make_map(&c->tm_q64, c->q, M, NQH * HD, 64) && make_map_f32(&c->tmo_qkv, c->acc_qkv, M, 2560, 128, false) &&
+            make_map_f32(&c->tmo_h, c->h, M, D, 128, false) && make_map_f32(&c->tmo_gu, c->acc_gu, M, 2 * F, 128, false);
   if (c->cfg.has_prefill) {
     ok = ok && make_map(&c->tm_pwqkv, c->pw_qkv, (uint64_t)L * 2560, DP, 128) &&
          make_map(&c->tm_pwo, c->pw_o, (uint64_t)L * DP, NQH * HD, 128) &&
          make_map(&c->tm_pwgu, c->pw_gu, (uint64_t)L * 2 * FP, DP, 128) &&
          make_map(&c->tm_pwd, c->pw_d, (uint64_t)L * DP, FP, 128) &&
          make_xmaps(&c->tm_pop, c->pop, Mp, DP) && make_xmaps(&c->tm_po, c->po, Mp, NQH * HD) &&
-         make_xmaps(&c->tm_pmb, c->pmb, Mp, FP);
+         make_xmaps(&c->tm_pmb, c->pmb, Mp, FP) && make_map_f32(&c->tmo_pqkv, c->pacc, Mp, 2560, 128, false) &&
+         make_map_f32(&c->tmo_px, c->px, Mp, DP, 128, false) && make_map_f32(&c->tmo_pgu, c->pacc, Mp, 2 * FP, 128, false);
   }
   if (!ok) return RTVLA_ERR_CUDA;
 
