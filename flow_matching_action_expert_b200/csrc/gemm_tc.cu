@@ -41,8 +41,10 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * 128;
-  const int m0 = blockIdx.y * TN;
+  // token tiles vary fastest, so the CTAs that share a weight tile run together and all but
+  // the first find it in L2
+  const int m0 = blockIdx.x * TN;
+  const int n0 = blockIdx.y * 128;
   const int kb_total = p.K >> 6;
   const int kb0 = blockIdx.z * p.kb_per_split;
   const int nkb = min(p.kb_per_split, kb_total - kb0);
@@ -146,7 +148,7 @@ template <int TN>
 static cudaError_t launch_tn(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmO,
                              const GemmParams &p, int n_tiles, int m_tiles, int splits, cudaStream_t st) {
   using G = GemmCfg<TN>;
-  dim3 grid(n_tiles, m_tiles, splits);
+  dim3 grid(m_tiles, n_tiles, splits);
   k_gemm_tc<TN><<<grid, 192, G::SMEM, st>>>(tmW, tmX, tmO, p);
   return cudaGetLastError();
 }
