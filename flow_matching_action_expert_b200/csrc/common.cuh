@@ -218,6 +218,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
                "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
+// wait until at most N committed bulk groups are still reading their shared-memory source
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // the shared source of every committed bulk operation has been read
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

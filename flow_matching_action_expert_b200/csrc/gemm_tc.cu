@@ -23,11 +23,34 @@ struct GemmCfg {
   static constexpr int W_BYTES = 128 * 128;  // 128 rows x 64 bf16
   static constexpr int X_BYTES = TN * 128;   // TN rows x 64 bf16
   static constexpr int STAGE = W_BYTES + X_BYTES;
-  static constexpr int STAGES = (TN <= 64) ? 8 : (TN <= 128 ? 6 : 4);
-  static constexpr int TMEM_COLS = TN <= 32 ? 32 : (TN <= 64 ? 64 : (TN <= 128 ? 128 : 256));
-  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr int STAGES = (TN <= 64) ? 6 : (TN <= 128 ? 5 : 3);
+  static constexpr int EPI = 64 * 128 * 4;   // one 64-token x 128-feature fp32 epilogue box
+  static constexpr int TMEM_COLS = 2 * (TN <= 32 ? 32 : TN);  // two accumulators
+  static constexpr int SMEM = STAGES * STAGE + 2 * EPI + 1024 + 256;
+  static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
+// Tile t of the launch: token tile t % m_tiles, weight tile (t / m_tiles) % n_tiles, K split
+// t / (m_tiles * n_tiles).  Token tiles vary fastest so the CTAs that share a weight tile run
+// together and all but the first find it in L2.
+struct TileIdx {
+  int m0, n0, kb0, nkb;
+};
+template <int TN>
+__device__ __forceinline__ TileIdx tile_at(const GemmParams &p, int t) {
+  TileIdx r;
+  const int mi = t % p.m_tiles, rest = t / p.m_tiles;
+  r.m0 = mi * TN;
+  r.n0 = (rest % p.n_tiles) * 128;
+  r.kb0 = (rest / p.n_tiles) * p.kb_per_split;
+  r.nkb = min(p.kb_per_split, (p.K >> 6) - r.kb0);
+  return r;
+}
+
+// Persistent: CTA c computes tiles c, c + grid, ...  Warp roles: warp 0 = TMA producer
+// through a STAGES-deep ring, warp 1 = MMA issuer alternating between two TMEM accumulators,
+// warps 2..5 = epilogue, which drains one accumulator (64 tokens at a time through two
+// shared-memory boxes and TMA bulk reduce / store) while the MMA fills the other.
 template <int TN>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -35,29 +58,29 @@ __global__ void __launch_bounds__(192, 1)
   using G = GemmCfg<TN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + G::STAGES * G::STAGE);
+  float *epi = reinterpret_cast<float *>(smem + G::STAGES * G::STAGE);  // [2][64][128]
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + G::STAGES * G::STAGE + 2 * G::EPI);
   uint64_t *empty = full + G::STAGES;
-  uint64_t *done = empty + G::STAGES;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  uint64_t *acc_full = empty + G::STAGES;  // [2]
+  uint64_t *acc_empty = acc_full + 2;      // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // token tiles vary fastest, so the CTAs that share a weight tile run together and all but
-  // the first find it in L2
-  const int m0 = blockIdx.x * TN;
-  const int n0 = blockIdx.y * 128;
-  const int kb_total = p.K >> 6;
-  const int kb0 = blockIdx.z * p.kb_per_split;
-  const int nkb = min(p.kb_per_split, kb_total - kb0);
+  const int ntiles = p.m_tiles * p.n_tiles * p.splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < G::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 1);
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, G::TMEM_COLS);
@@ -69,71 +92,105 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0 && nkb > 0) {
+    if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % G::STAGES;
-        const uint32_t ph = (i / G::STAGES) & 1;
-        if (i >= G::STAGES && !mbar_wait(&empty[s], ph ^ 1, p.ctl, 101)) break;
-        uint8_t *st = smem + s * G::STAGE;
-        mbar_arrive_expect_tx(&full[s], G::STAGE);
-        tma_load_2d(st, &tmW, &full[s], (kb0 + i) * 64, p.w_row0 + n0, pol_w);
-        tma_load_2d(st + G::W_BYTES, &tmX, &full[s], (kb0 + i) * 64, m0, pol_x);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const TileIdx ti = tile_at<TN>(p, t);
+        for (int i = 0; i < ti.nkb; ++i, ++it) {
+          const int s = it % G::STAGES;
+          if (it >= (uint32_t)G::STAGES && !mbar_wait(&empty[s], ((it / G::STAGES) & 1) ^ 1, p.ctl, 101)) {
+            ok = false;
+            break;
+          }
+          uint8_t *st = smem + s * G::STAGE;
+          mbar_arrive_expect_tx(&full[s], G::STAGE);
+          tma_load_2d(st, &tmW, &full[s], (ti.kb0 + i) * 64, p.w_row0 + ti.n0, pol_w);
+          tma_load_2d(st + G::W_BYTES, &tmX, &full[s], (ti.kb0 + i) * 64, ti.m0, pol_x);
+        }
       }
+      // every issued copy must land before the CTA may exit
+      const uint32_t first = it > (uint32_t)G::STAGES ? it - G::STAGES : 0;
+      for (uint32_t j = first; j < it; ++j) mbar_wait(&full[j % G::STAGES], (j / G::STAGES) & 1, p.ctl, 104);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, TN);
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % G::STAGES;
-        const uint32_t ph = (i / G::STAGES) & 1;
-        if (!mbar_wait(&full[s], ph, p.ctl, 102)) break;
+      uint32_t it = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++local) {
+        const TileIdx ti = tile_at<TN>(p, t);
+        const int b = local & 1;
+        // the epilogue must have drained this accumulator (used two tiles ago)
+        if (local >= 2 && !mbar_wait(&acc_empty[b], ((local >> 1) & 1) ^ 1, p.ctl, 105)) break;
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + s * G::STAGE);
-        const uint32_t b = a + G::W_BYTES;
+        const uint32_t d = tmem + (uint32_t)(b * (G::TMEM_COLS / 2));
+        for (int i = 0; i < ti.nkb; ++i, ++it) {
+          const int s = it % G::STAGES;
+          if (!mbar_wait(&full[s], (it / G::STAGES) & 1, p.ctl, 102)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + s * G::STAGE);
+          const uint32_t bx = a + G::W_BYTES;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tmem, sdesc_k128(a + 32 * k), sdesc_k128(b + 32 * k), idesc, (i > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&empty[s]);
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(d, sdesc_k128(a + 32 * k), sdesc_k128(bx + 32 * k), idesc, (i > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&acc_full[b]);
       }
-      umma_commit(done);
     }
-  } else if (nkb > 0) {
-    // epilogue: warp (2..5) & 3 selects the TMEM lane quadrant it may access; the tile reuses
-    // the pipeline stages (every TMA load into them has been consumed once `done` fires)
-    static_assert(TN * 128 * 4 <= G::STAGES * G::STAGE, "epilogue tile fits the stages");
-    float *tile = reinterpret_cast<float *>(smem);
+  } else {
+    // epilogue: warp (2..5) & 3 selects the TMEM lane quadrant (features) it may access
     const int q = warp & 3;
     const int nl = q * 32 + lane;
-    if (mbar_wait(done, 0, p.ctl, 103)) {
+    const bool leader = warp == 2 && lane == 0;
+    int local = 0;
+    uint32_t nbox = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+      const TileIdx ti = tile_at<TN>(p, t);
+      const int b = local & 1;
+      if (!mbar_wait(&acc_full[b], (local >> 1) & 1, p.ctl, 103)) break;
       tc_fence_after();
-      const float sc = p.col_scale ? p.col_scale[n0 + nl] : 1.0f;
+      const uint32_t d = tmem + (uint32_t)(b * (G::TMEM_COLS / 2)) + ((uint32_t)(q * 32) << 16);
+      const float sc = p.col_scale ? p.col_scale[ti.n0 + nl] : 1.0f;
+      for (int c0 = 0; c0 < TN && ti.m0 + c0 < p.M; c0 += 64, ++nbox) {
+        float *box = epi + (nbox & 1) * (64 * 128);
+        if (leader && nbox >= 2) bulk_wait_read<1>();  // the copy that last read this box is done
+        asm volatile("bar.sync 1, 128;" ::: "memory");
 #pragma unroll 1
-      for (int c = 0; c < TN; c += 32) {
-        float v[32];
-        if (m0 + c < p.M) {
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-        } else {
+        for (int c = c0; c < c0 + 64 && c < TN; c += 32) {
+          float v[32];
+          if (ti.m0 + c < p.M) {
+            tmem_ld32(d + (uint32_t)c, v);
+          } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) box[(c - c0 + j) * 128 + nl] = (ti.m0 + c + j < p.M) ? v[j] * sc : 0.f;
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) tile[(c + j) * 128 + nl] = (m0 + c + j < p.M) ? v[j] * sc : 0.f;
+        fence_proxy_async_shared();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (leader) {
+          if (p.atomic)
+            tma_reduce_add_2d(&tmO, box, ti.n0, ti.m0 + c0);
+          else
+            tma_store_2d(&tmO, box, ti.n0, ti.m0 + c0);
+          bulk_commit();
+        }
       }
+      // the accumulator has been read: hand it back to the MMA issuer
+      tc_fence_before();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (leader) mbar_arrive(&acc_empty[b]);
     }
-    fence_proxy_async_shared();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (warp == 2 && lane == 0) {
-      for (int t = 0; t < TN && m0 + t < p.M; t += 64) {
-        if (p.atomic)
-          tma_reduce_add_2d(&tmO, tile + t * 128, n0, m0 + t);
-        else
-          tma_store_2d(&tmO, tile + t * 128, n0, m0 + t);
-      }
-      bulk_commit();
-      bulk_wait_read0();  // the tile must stay valid until the bulk copies have read it
-    }
+    if (leader) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -146,10 +203,10 @@ __global__ void __launch_bounds__(192, 1)
 
 template <int TN>
 static cudaError_t launch_tn(const CUtensorMap &tmW, const CUtensorMap &tmX, const CUtensorMap &tmO,
-                             const GemmParams &p, int n_tiles, int m_tiles, int splits, cudaStream_t st) {
+                             const GemmParams &p, int sm_count, cudaStream_t st) {
   using G = GemmCfg<TN>;
-  dim3 grid(m_tiles, n_tiles, splits);
-  k_gemm_tc<TN><<<grid, 192, G::SMEM, st>>>(tmW, tmX, tmO, p);
+  const int tiles = p.m_tiles * p.n_tiles * p.splits;
+  k_gemm_tc<TN><<<dim3(tiles < sm_count ? tiles : sm_count), 192, G::SMEM, st>>>(tmW, tmX, tmO, p);
   return cudaGetLastError();
 }
 
@@ -198,11 +255,14 @@ cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int
   p.col_scale = col_scale;
   p.atomic = (accumulate || g.splits > 1) ? 1 : 0;
   p.ctl = ctl;
+  p.m_tiles = g.m_tiles;
+  p.n_tiles = g.n_tiles;
+  p.splits = g.splits;
   const CUtensorMap &tmX = xm.m[gemm_tile_index(g.tn)];
   switch (g.tn) {
-    case 64: return launch_tn<64>(tmW, tmX, tmO, p, g.n_tiles, g.m_tiles, g.splits, st);
-    case 128: return launch_tn<128>(tmW, tmX, tmO, p, g.n_tiles, g.m_tiles, g.splits, st);
-    default: return launch_tn<256>(tmW, tmX, tmO, p, g.n_tiles, g.m_tiles, g.splits, st);
+    case 64: return launch_tn<64>(tmW, tmX, tmO, p, sm_count, st);
+    case 128: return launch_tn<128>(tmW, tmX, tmO, p, sm_count, st);
+    default: return launch_tn<256>(tmW, tmX, tmO, p, sm_count, st);
   }
 }
 

@@ -20,6 +20,7 @@ struct GemmParams {
   const float *col_scale;  // per-output-column factor (AdaRMS gate) or null
   int atomic;              // 1: fp32 reduction into out; 0: plain store
   DevCtl *ctl;
+  int m_tiles, n_tiles, splits;  // the launch's tiles (a CTA loops over tile c, c + grid, ...)
 };
 
 struct GemmPlan {
