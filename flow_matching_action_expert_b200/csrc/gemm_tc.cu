@@ -219,7 +219,7 @@ cudaError_t gemm_init_attributes() {
   return e;
 }
 
-// Chooses the token tile and the K split so that about one wave of 148 SMs is busy.
+// Chooses the token tile and the K split (at most one round of tiles over the SMs).
 GemmPlan gemm_plan(int M, int N, int K, int sm_count) {
   GemmPlan g;
   // a 128 x 256 x 16 MMA costs about as much as 128 x 128 x 16 (and 128 x 64 x 16) on sm_100a,
@@ -229,7 +229,9 @@ GemmPlan gemm_plan(int M, int N, int K, int sm_count) {
   g.n_tiles = N / 128;
   const int kb_total = K / 64;
   const int units = g.n_tiles * g.m_tiles;
-  int splits = (sm_count + units - 1) / units;
+  // split K only as far as one round of tiles fits the SMs: a second, partial round would cost
+  // a whole tile time, and splits beyond that only add reduction traffic
+  int splits = sm_count / units;
   if (splits < 1) splits = 1;
   if (splits > kb_total) splits = kb_total;
   g.kb_per_split = (kb_total + splits - 1) / splits;
