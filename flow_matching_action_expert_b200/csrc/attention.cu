@@ -45,15 +45,24 @@ __global__ void __launch_bounds__(256, 1) k_attn(AttnParams p) {
   const int k_begin = split * p.keys_per_split;
   const int k_end = min(total, k_begin + p.keys_per_split);
 
-  // stage the 16 x 8 query rows
-  for (int idx = threadIdx.x; idx < NH * QB * (HD / 8); idx += 256) {
-    const int c8 = idx % (HD / 8);
-    const int row = (idx / (HD / 8)) % QB;
-    const int h = idx / (QB * (HD / 8));
-    const int qi = qb * QB + row;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (qi < p.nq) v = *reinterpret_cast<const uint4 *>(p.q + (size_t)(b * p.nq + qi) * p.q_ld + h * HD + c8 * 8);
-    *reinterpret_cast<uint4 *>(Qs + (h * QB + row) * LDS + c8 * 8) = v;
+  // stage the 16 x 8 query rows: all of a thread's loads in flight before its stores
+  {
+    constexpr int NQL = NH * QB * (HD / 8) / 256;
+    uint4 qv[NQL];
+#pragma unroll
+    for (int i = 0; i < NQL; ++i) {
+      const int idx = threadIdx.x + i * 256;
+      const int c8 = idx % (HD / 8), row = (idx / (HD / 8)) % QB, h = idx / (QB * (HD / 8));
+      const int qi = qb * QB + row;
+      qv[i] = qi < p.nq ? *reinterpret_cast<const uint4 *>(p.q + (size_t)(b * p.nq + qi) * p.q_ld + h * HD + c8 * 8)
+                        : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < NQL; ++i) {
+      const int idx = threadIdx.x + i * 256;
+      const int c8 = idx % (HD / 8), row = (idx / (HD / 8)) % QB, h = idx / (QB * (HD / 8));
+      *reinterpret_cast<uint4 *>(Qs + (h * QB + row) * LDS + c8 * 8) = qv[i];
+    }
   }
 
   float o[32][4];
@@ -65,22 +74,31 @@ __global__ void __launch_bounds__(256, 1) k_attn(AttnParams p) {
 
 #pragma unroll 1
   for (int c0 = k_begin; c0 < k_end; c0 += KC) {
-    __syncthreads();  // previous chunk fully consumed (and Q staged on the first pass)
-    for (int idx = threadIdx.x; idx < KC * (HD / 8); idx += 256) {
-      const int c8 = idx % (HD / 8);
-      const int r = idx / (HD / 8);
-      const int j = c0 + r;
-      uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+    // this chunk's K / V rows: every load of the thread in flight before any store (the
+    // prefix rows come from HBM; one round trip instead of eight)
+    constexpr int NKL = KC * (HD / 8) / 256;
+    uint4 kv[NKL], vv[NKL];
+#pragma unroll
+    for (int i = 0; i < NKL; ++i) {
+      const int idx = threadIdx.x + i * 256;
+      const int c8 = idx % (HD / 8), j = c0 + idx / (HD / 8);
+      kv[i] = vv[i] = make_uint4(0, 0, 0, 0);
       if (j < lv) {
-        kv = *reinterpret_cast<const uint4 *>(kpre + (size_t)j * HD + c8 * 8);
-        vv = *reinterpret_cast<const uint4 *>(vpre + (size_t)j * HD + c8 * 8);
+        kv[i] = *reinterpret_cast<const uint4 *>(kpre + (size_t)j * HD + c8 * 8);
+        vv[i] = *reinterpret_cast<const uint4 *>(vpre + (size_t)j * HD + c8 * 8);
       } else if (j < k_end) {
         const size_t off = ((size_t)b * p.n_suf + (j - lv)) * HD + c8 * 8;
-        kv = *reinterpret_cast<const uint4 *>(p.ksuf + off);
-        vv = *reinterpret_cast<const uint4 *>(p.vsuf + off);
+        kv[i] = *reinterpret_cast<const uint4 *>(p.ksuf + off);
+        vv[i] = *reinterpret_cast<const uint4 *>(p.vsuf + off);
       }
-      *reinterpret_cast<uint4 *>(Ks + r * LDS + c8 * 8) = kv;
-      *reinterpret_cast<uint4 *>(Vs + r * LDS + c8 * 8) = vv;
+    }
+    __syncthreads();  // previous chunk fully consumed (and Q staged on the first pass)
+#pragma unroll
+    for (int i = 0; i < NKL; ++i) {
+      const int idx = threadIdx.x + i * 256;
+      const int c8 = idx % (HD / 8), r = idx / (HD / 8);
+      *reinterpret_cast<uint4 *>(Ks + r * LDS + c8 * 8) = kv[i];
+      *reinterpret_cast<uint4 *>(Vs + r * LDS + c8 * 8) = vv[i];
     }
     __syncthreads();
 
