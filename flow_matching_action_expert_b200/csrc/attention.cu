@@ -221,11 +221,13 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnParams p) {
   const int b = row / p.nq, i = row % p.nq;
   const int h = threadIdx.x >> 5, d0 = (threadIdx.x & 31) * 8;
   float M = -INFINITY;
+#pragma unroll 4
   for (int s = 0; s < p.n_splits; ++s)
     M = fmaxf(M, p.mlpart[((((size_t)b * p.n_splits + s) * p.nq + i) * NH + h) * 2]);
   const float ref = (M == -INFINITY) ? 0.f : M;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   float L = 0.f;
+#pragma unroll 4
   for (int s = 0; s < p.n_splits; ++s) {
     const size_t r = (((size_t)b * p.n_splits + s) * p.nq + i) * NH + h;
     const float2 ml = *reinterpret_cast<const float2 *>(p.mlpart + r * 2);

@@ -69,10 +69,15 @@ __global__ void __launch_bounds__(256) k_adanorm(const float *h, const float *s1
 }
 
 // QKV epilogue: y = r * acc + bias; RoPE (pairs d, d+128) at position Lv_b + j on the 8 query
-// heads and the key; Q -> [M][2048], K_s, V_s -> [M][256] (bf16).  Clears acc.
-__global__ void __launch_bounds__(256) k_qkv_post(float *acc, const float *r, const float *bias, const CallArgs *ca,
-                                                  int C, const float *rc, const float *rs, int rope_rows, bf16 *q,
-                                                  bf16 *ks, bf16 *vs, DevCtl *ctl) {
+// heads and the key; Q -> [M][2048], K_s, V_s -> [M][256] (bf16).  Clears acc.  Thread t owns
+// 4 consecutive d of the rotated pairs in one head (288 pair groups: 8 query heads + the key,
+// 32 per head) and, for t < 64, 4 consecutive columns of V; every load is issued before any
+// store.
+__global__ void __launch_bounds__(256) k_qkv_post(float *__restrict__ acc, const float *__restrict__ r,
+                                                  const float *__restrict__ bias, const CallArgs *ca, int C,
+                                                  const float *__restrict__ rc, const float *__restrict__ rs,
+                                                  int rope_rows, bf16 *__restrict__ q, bf16 *__restrict__ ks,
+                                                  bf16 *__restrict__ vs, DevCtl *ctl) {
   const int m = blockIdx.x;
   const int b = m / C, j = m % C;
   int pos = ca->valid_len[b] + j;
@@ -82,48 +87,94 @@ __global__ void __launch_bounds__(256) k_qkv_post(float *acc, const float *r, co
   }
   float *a = acc + (size_t)m * 2560;
   const float rr = r[m];
-  const float *cr = rc + (size_t)pos * 128;
-  const float *sr = rs + (size_t)pos * 128;
-  for (int i = threadIdx.x; i < 9 * 128; i += 256) {
-    const int head = i >> 7, d = i & 127;
-    const int c1 = head * 256 + d, c2 = c1 + 128;
-    const float x1 = rr * a[c1] + bias[c1];
-    const float x2 = rr * a[c2] + bias[c2];
-    const float co = cr[d], si = sr[d];
-    const float y1 = x1 * co - x2 * si;
-    const float y2 = x2 * co + x1 * si;
-    if (head < 8) {
-      q[(size_t)m * 2048 + c1] = f2bf(y1);
-      q[(size_t)m * 2048 + c2] = f2bf(y2);
-    } else {
-      ks[(size_t)m * 256 + d] = f2bf(y1);
-      ks[(size_t)m * 256 + d + 128] = f2bf(y2);
-    }
+  // two pair groups per thread (the first 32 threads take a third), loaded together
+  float4 x1[2], x2[2], b1[2], b2[2], co[2], si[2];
+  int grp[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    grp[k] = threadIdx.x + k * 256;
+    const int g = grp[k] < 288 ? grp[k] : 0;
+    const int head = g >> 5, d = (g & 31) * 4;
+    const int c1 = head * 256 + d;
+    x1[k] = *reinterpret_cast<const float4 *>(a + c1);
+    x2[k] = *reinterpret_cast<const float4 *>(a + c1 + 128);
+    b1[k] = *reinterpret_cast<const float4 *>(bias + c1);
+    b2[k] = *reinterpret_cast<const float4 *>(bias + c1 + 128);
+    co[k] = *reinterpret_cast<const float4 *>(rc + (size_t)pos * 128 + d);
+    si[k] = *reinterpret_cast<const float4 *>(rs + (size_t)pos * 128 + d);
   }
-  for (int d = threadIdx.x; d < 256; d += 256) vs[(size_t)m * 256 + d] = f2bf(rr * a[2304 + d] + bias[2304 + d]);
-  __syncthreads();
+  float4 vx = make_float4(0, 0, 0, 0), vb = vx;
+  if (threadIdx.x < 64) {
+    vx = *reinterpret_cast<const float4 *>(a + 2304 + threadIdx.x * 4);
+    vb = *reinterpret_cast<const float4 *>(bias + 2304 + threadIdx.x * 4);
+  }
+  __syncthreads();  // every read of this row's accumulator is done before it is cleared
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    if (grp[k] >= 288) continue;
+    const int head = grp[k] >> 5, d = (grp[k] & 31) * 4;
+    const float *u = reinterpret_cast<const float *>(&x1[k]), *w = reinterpret_cast<const float *>(&x2[k]);
+    const float *bu = reinterpret_cast<const float *>(&b1[k]), *bw = reinterpret_cast<const float *>(&b2[k]);
+    const float *cs = reinterpret_cast<const float *>(&co[k]), *sn = reinterpret_cast<const float *>(&si[k]);
+    float y1[4], y2[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float p1 = rr * u[e] + bu[e], p2 = rr * w[e] + bw[e];
+      y1[e] = p1 * cs[e] - p2 * sn[e];
+      y2[e] = p2 * cs[e] + p1 * sn[e];
+    }
+    bf16 *dst = head < 8 ? q + (size_t)m * 2048 + head * 256 : ks + (size_t)m * 256;
+    uint2 lo, hi;
+    lo.x = pack_bf16(y1[0], y1[1]);
+    lo.y = pack_bf16(y1[2], y1[3]);
+    hi.x = pack_bf16(y2[0], y2[1]);
+    hi.y = pack_bf16(y2[2], y2[3]);
+    *reinterpret_cast<uint2 *>(dst + d) = lo;
+    *reinterpret_cast<uint2 *>(dst + d + 128) = hi;
+  }
+  if (threadIdx.x < 64) {
+    uint2 o;
+    o.x = pack_bf16(rr * vx.x + vb.x, rr * vx.y + vb.y);
+    o.y = pack_bf16(rr * vx.z + vb.z, rr * vx.w + vb.w);
+    *reinterpret_cast<uint2 *>(vs + (size_t)m * 256 + threadIdx.x * 4) = o;
+  }
   for (int i = threadIdx.x; i < 2560 / 4; i += 256) reinterpret_cast<float4 *>(a)[i] = make_float4(0, 0, 0, 0);
 }
 
 // out[m][j] = bf16(GELU_tanh(r*g + bg) * (r*u + bu)), g = acc[m][j], u = acc[m][F + j].  Clears acc.
-__global__ void __launch_bounds__(256) k_gelu_mul(float *acc, const float *r, const float *bias, bf16 *out, int F) {
+// Every load of a thread (F / 1024 groups of 4 columns) is issued before any store.
+__global__ void __launch_bounds__(256) k_gelu_mul(float *__restrict__ acc, const float *__restrict__ r,
+                                                  const float *__restrict__ bias, bf16 *__restrict__ out, int F) {
   const int m = blockIdx.x;
   float *a = acc + (size_t)m * 2 * F;
   const float rr = r ? r[m] : 1.0f;
-  for (int j = threadIdx.x * 4; j < F; j += 1024) {
-    float4 g = *reinterpret_cast<float4 *>(a + j);
-    float4 u = *reinterpret_cast<float4 *>(a + F + j);
-    float4 bg = make_float4(0, 0, 0, 0), bu = bg;
-    if (bias) {
-      bg = *reinterpret_cast<const float4 *>(bias + j);
-      bu = *reinterpret_cast<const float4 *>(bias + F + j);
+  const int ng = F / 1024;
+#pragma unroll 1
+  for (int g0 = 0; g0 < ng; g0 += 4) {
+    float4 g[4], u[4], bg[4], bu[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = (g0 + k) * 1024 + threadIdx.x * 4;
+      if (g0 + k < ng) {
+        g[k] = *reinterpret_cast<const float4 *>(a + j);
+        u[k] = *reinterpret_cast<const float4 *>(a + F + j);
+        bg[k] = bias ? *reinterpret_cast<const float4 *>(bias + j) : make_float4(0, 0, 0, 0);
+        bu[k] = bias ? *reinterpret_cast<const float4 *>(bias + F + j) : make_float4(0, 0, 0, 0);
+      }
     }
-    uint2 o;
-    o.x = pack_bf16(gelu_tanh(rr * g.x + bg.x) * (rr * u.x + bu.x), gelu_tanh(rr * g.y + bg.y) * (rr * u.y + bu.y));
-    o.y = pack_bf16(gelu_tanh(rr * g.z + bg.z) * (rr * u.z + bu.z), gelu_tanh(rr * g.w + bg.w) * (rr * u.w + bu.w));
-    *reinterpret_cast<uint2 *>(out + (size_t)m * F + j) = o;
-    *reinterpret_cast<float4 *>(a + j) = make_float4(0, 0, 0, 0);
-    *reinterpret_cast<float4 *>(a + F + j) = make_float4(0, 0, 0, 0);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (g0 + k >= ng) break;
+      const int j = (g0 + k) * 1024 + threadIdx.x * 4;
+      uint2 o;
+      o.x = pack_bf16(gelu_tanh(rr * g[k].x + bg[k].x) * (rr * u[k].x + bu[k].x),
+                      gelu_tanh(rr * g[k].y + bg[k].y) * (rr * u[k].y + bu[k].y));
+      o.y = pack_bf16(gelu_tanh(rr * g[k].z + bg[k].z) * (rr * u[k].z + bu[k].z),
+                      gelu_tanh(rr * g[k].w + bg[k].w) * (rr * u[k].w + bu[k].w));
+      *reinterpret_cast<uint2 *>(out + (size_t)m * F + j) = o;
+      *reinterpret_cast<float4 *>(a + j) = make_float4(0, 0, 0, 0);
+      *reinterpret_cast<float4 *>(a + F + j) = make_float4(0, 0, 0, 0);
+    }
   }
 }
 
