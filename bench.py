@@ -98,6 +98,18 @@ def algorithmic(wl):
     return bytes_step * S, flops_step * S, w_bytes * S
 
 
+def reduce_max(vals, device):
+    """Each value's maximum over the ranks of the current process group (a replica job takes
+    as long as its slowest rank); the values themselves without a group or with one rank."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -289,11 +301,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = statistics.mean(per)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max([statistics.mean(per)], dev)[0]
     st = R.rtvla_sync_status(ctx, stream)
     if st != 0:
         raise RuntimeError(f"device status {R.STATUS[st]}")
@@ -316,11 +324,7 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         e1.synchronize()
         e2e.append(e0.elapsed_time(e1))
-    e2e_ms = statistics.mean(e2e)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max([statistics.mean(e2e)], dev)[0]
     h2d = hn.numel() * 4 + hk.numel() * 2 + hv.numel() * 2 + hl.numel() * 4
     d2h = ho.numel() * 4
     R.rtvla_destroy(ctx)
@@ -432,11 +436,7 @@ def run_e2e(args, rank, world, local_rank, wl):
     pre = [a.elapsed_time(b) for a, b, _ in ev]
     den = [b.elapsed_time(c) for _, b, c in ev]
     tot = [a.elapsed_time(c) for a, _, c in ev]
-    ms, pre_ms, den_ms = statistics.mean(tot), statistics.mean(pre), statistics.mean(den)
-    if world > 1:
-        t = torch.tensor([ms, pre_ms, den_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, pre_ms, den_ms = (float(x) for x in t.tolist())
+    ms, pre_ms, den_ms = reduce_max([statistics.mean(tot), statistics.mean(pre), statistics.mean(den)], dev)
     st = R.rtvla_sync_status(ctx, stream)
     if st != 0:
         raise RuntimeError(f"device status {R.STATUS[st]}")
