@@ -65,6 +65,16 @@ def workload(batch, name="2-view"):
     return WL.workload(3) if batch == 1 else WL.workload(4, batch=batch)
 
 
+def workload_config(wl, world):
+    """The `config` object of the JSON line: the workload only, the same on both arms."""
+    c = {"workload": wl.name, "batch": wl.batch, "chunk": wl.chunk, "prefix": wl.prefix_cap,
+         "valid_prefix": list(wl.valid_lens)[:4], "layers": wl.expert.n_layers,
+         "steps_per_loop": wl.expert.n_steps, "parallelism": f"replicas{world}"}
+    if wl.prefill is not None:
+        c["prefill_layers"] = wl.prefill.n_layers
+    return c
+
+
 def prefill_algorithmic(wl):
     """Bytes and FLOPs of one prefill pass: every layer's weights read once; 2 * T * params plus
     the bidirectional attention over the valid prefix; the last layer computes K and V only."""
@@ -239,8 +249,8 @@ def run_reference(args, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_loop, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, N(0,1) KV and noise)",
-        "config": {"workload": wl.name, "batch": wl.batch, "chunk": wl.chunk, "prefix": wl.prefix_cap,
-                   "layers": wl.expert.n_layers, "steps_per_loop": wl.expert.n_steps},
+        "config": workload_config(wl, args.gpus),
+        "engine": "oracle (fp64 numpy, host cores)",
         "cpu_baseline": {"value": round(per_loop, 3), "unit": "ms", "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"{len(times)} x one Euler step of the loop (fp64 oracle, S=1), x10 per loop"},
         "e2e": {"value": round(per_loop, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -344,10 +354,9 @@ def run_ours(args, rank, world, local_rank):
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, N(0,1) KV and noise)",
-        "config": {"workload": wl.name, "batch": wl.batch, "chunk": wl.chunk, "prefix": wl.prefix_cap,
-                   "valid_prefix": list(wl.valid_lens)[:4], "layers": wl.expert.n_layers,
-                   "steps_per_loop": wl.expert.n_steps, "engine": engine, "parallelism": f"replicas{world}",
-                   "l2": "flushed by a 256 MiB write between timed loops; weights (623 MB) exceed L2"},
+        "config": workload_config(wl, world),
+        "engine": engine,
+        "l2": "flushed by a 256 MiB write between timed loops; weights (623 MB) exceed L2",
         "hbm_gbs_achieved": round(achieved_gbs, 1),
         "chunks_per_s": round(world * wl.batch / (ms * 1e-3), 2),
         "latency_ms": {"p10": round(float(np.percentile(per, 10)), 4), "p50": round(float(np.median(per)), 4),
@@ -455,10 +464,8 @@ def run_e2e(args, rank, world, local_rank, wl):
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, N(0,1)*sqrt(2048) prefix embeddings, N(0,1) noise)",
-        "config": {"workload": wl.name, "batch": wl.batch, "chunk": wl.chunk, "prefix": wl.prefix_cap,
-                   "prefill_layers": wl.prefill.n_layers, "layers": wl.expert.n_layers,
-                   "steps_per_loop": wl.expert.n_steps, "parallelism": f"replicas{world}",
-                   "l2": "flushed by a 256 MiB write between timed steps; weights (4.4 GB) exceed L2"},
+        "config": workload_config(wl, world),
+        "l2": "flushed by a 256 MiB write between timed steps; weights (4.4 GB) exceed L2",
         "prefill_ms": round(pre_ms, 4), "denoise_ms": round(den_ms, 4),
         "roofline": {"bound": "tensor", "kernel": "rtvla_prefill (layered tcgen05 GEMMs + attention)",
                      "achieved": round(pf / (pre_ms * 1e-3) / 1e12, 1), "peak": bf16_sus, "unit": "TFLOP/s",
