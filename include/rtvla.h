@@ -49,11 +49,16 @@ typedef enum {
   RTVLA_ERR_DEVICE_BOUNDS = 8    /* a valid length exceeded its buffer (device-detected, clamped) */
 } rtvla_status;
 
-/* Engines that run the denoise loop (rtvla_config.engine). */
+/* Engines that run the denoise loop (rtvla_config.engine).  The persistent engine applies to
+ * calls with batch 1 and chunk <= 64 on a GPU where its cooperative launch fits (one CTA of
+ * 320 threads and ~218 KB of shared memory per SM, >= 64 SMs; rtvla_kernels_per_call then
+ * returns 1).  Results of the two engines agree within the parity tolerance, not bitwise
+ * (split-K sums are reduced in a different order). */
 enum {
-  RTVLA_ENGINE_AUTO = 0,       /* persistent kernel when it applies, else layered */
+  RTVLA_ENGINE_AUTO = 0,       /* the persistent kernel when it applies, else layered */
   RTVLA_ENGINE_LAYERED = 1,    /* one kernel per phase, the whole loop captured as one CUDA graph */
-  RTVLA_ENGINE_PERSISTENT = 2  /* one persistent kernel per call that streams weights continuously */
+  RTVLA_ENGINE_PERSISTENT = 2  /* one persistent kernel per call; calls it cannot serve return
+                                  RTVLA_ERR_UNSUPPORTED */
 };
 
 /*
