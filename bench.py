@@ -171,12 +171,38 @@ class Clocks:
 KERNEL_SOURCES = ("csrc/persistent.cu", "csrc/persistent.h", "csrc/common.cuh", "csrc/rtvla_api.cu")
 
 
+def strip_comments(src):
+    """C/C++ source without comments and with whitespace collapsed: what the compiler sees."""
+    import re
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif src[i] == '"':  # string literal (the asm templates), copied as is
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def kernel_source_hash():
+    """sha256 of the persistent kernel's sources with comments and whitespace removed, so a
+    recorded capture stays valid across comment edits and is invalidated by any code change."""
     import hashlib
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "flow_matching_action_expert_b200", rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "flow_matching_action_expert_b200", rel), encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode())
+        h.update(b"\0")
     return h.hexdigest()
 
 

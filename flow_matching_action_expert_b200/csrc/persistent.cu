@@ -4,12 +4,12 @@
 // The loop is weight-streaming bound (622 MB of bf16 expert weights per Euler step) and is
 // a chain of dependent phases per layer.  Weights never depend on activations, so:
 //   warp 0     TMA producer: walks this CTA's static list of weight tiles for every GEMM of
-//              the whole loop and keeps a 7-stage shared-memory ring full, never waiting on
-//              an activation;
+//              the whole loop and keeps a 5-stage shared-memory ring full, never waiting on
+//              an activation; it also prefetches the next phase's table slices into L2;
 //   warp 1     tcgen05 MMA issuer (accumulator in TMEM), started per 64-wide K block as soon
 //              as that block of the activation operand is in shared memory;
-//   warps 2..9 compute: stage activations with TMA (fp32 tiles, 128-byte swizzle) and turn
-//              them into the bf16 operand (fused AdaRMS modulation / GELU(gate) * up), run
+//   warps 2..9 compute: stage activations with TMA (fp32 tiles, 128-byte swizzle, four
+//              per 3-D box) and turn them into the bf16 operand (fused AdaRMS modulation / GELU(gate) * up), run
 //              the epilogue (TMEM -> shared tile -> one TMA bulk reduce-add into fp32; the
 //              AdaRMS gate of the residual applied on the way), and run the Q/K/V finalise,
 //              attention, split merge and final / Euler phases; a grid barrier separates
