@@ -28,6 +28,18 @@ Readings where the pages are silent or ambiguous (each is also listed in the des
   R10 GELU is the tanh approximation.
   R11 attention scaling 1/sqrt(head_dim), no soft-cap.
   R12 t_k = 1 - k/S evaluated exactly (not accumulated), dt = -1/S.
+
+The π0 variant (``pi0_sample_actions``) follows [PAPER-S] ("Running VLAs at Real-time
+Speed" summary, section "How": the action time encoder's two linears fold, and its 10
+timestep rows become a table in the bias before SiLU; "π0 preliminaries": the state and the
+noisy actions are routed to the action expert, a Gemma reduced in width).  Readings:
+  P1 suffix = [one state token ; C action tokens]; state token = Linear(32 -> width)(state).
+  P2 action token = Linear_out(SiLU(Linear_in([action_in_proj(x) ; SinEmb(t)]))): the time
+     embedding (R2) is concatenated to each projected action, then a 2-layer MLP.
+  P3 every norm is a plain Gemma RMSNorm, x_hat * (1 + w) (R8, R9); residuals are ungated.
+  P4 the C + 1 suffix tokens attend to every valid prefix key and to each other (as R6),
+     at positions Lv + i, i = 0 for the state token (as R5).
+  P5 a final RMSNorm, then action_out_proj on the C action tokens only; Euler as R12.
 """
 from __future__ import annotations
 
@@ -281,3 +293,81 @@ def prefill(weights, cfg, embeds, pad_mask):
             n2 = rms_normalize(x, cfg.rms_eps) * (1.0 + W[p + "ln2"])
             x = x + (gelu_tanh(n2 @ W[p + "wg"].T) * (n2 @ W[p + "wu"].T)) @ W[p + "wd"].T
     return K, V, valid_len
+
+
+# ---------------------------------------------------------------------------------------
+# π0 suffix variant (readings P1-P5 in the header)
+
+def pi0_layer(h, W, l, k_pref, v_pref, lv, cfg):
+    """One π0 action-expert layer for one sample: plain RMSNorm (reading P3), attention over
+    [valid prefix ; all suffix tokens] (P4), ungated residuals.  h [T, D], T = C + 1."""
+    T, D = h.shape
+    H, hd, Hkv = cfg.n_q_heads, cfg.head_dim, cfg.n_kv_heads
+    P = k_pref.shape[0]
+    p = f"l{l}."
+    n = rms_normalize(h, cfg.rms_eps) * (1.0 + W[p + "ln1"])
+    q = (n @ W[p + "wq"].T).reshape(T, H, hd).transpose(1, 0, 2)
+    k = (n @ W[p + "wk"].T).reshape(T, Hkv, hd).transpose(1, 0, 2)
+    v = (n @ W[p + "wv"].T).reshape(T, Hkv, hd).transpose(1, 0, 2)
+    pos = lv + np.arange(T)
+    q = rope(q, pos, cfg.rope_theta)
+    k = rope(k, pos, cfg.rope_theta)
+    K = np.concatenate([np.broadcast_to(k_pref, (Hkv, P, hd)), k], axis=1)
+    V = np.concatenate([np.broadcast_to(v_pref, (Hkv, P, hd)), v], axis=1)
+    mask = np.zeros((T, P + T), dtype=bool)
+    mask[:, :lv] = True
+    mask[:, P:] = True
+    o = attention(q, K, V, mask, hd ** -0.5)
+    h = h + o.transpose(1, 0, 2).reshape(T, H * hd) @ W[p + "wo"].T
+    n2 = rms_normalize(h, cfg.rms_eps) * (1.0 + W[p + "ln2"])
+    return h + (gelu_tanh(n2 @ W[p + "wg"].T) * (n2 @ W[p + "wu"].T)) @ W[p + "wd"].T
+
+
+def pi0_suffix(W, x, state, t, cfg):
+    """The π0 suffix tokens [state ; actions] of one sample at time t (readings P1, P2)."""
+    a = x @ W["action_in_w"].T + W["action_in_b"]
+    e = sinusoidal_time_embedding(t, cfg.width)
+    at = np.concatenate([a, np.broadcast_to(e, a.shape)], axis=-1)
+    h_a = silu(at @ W["action_time_in_w"].T + W["action_time_in_b"]) @ W["action_time_out_w"].T \
+        + W["action_time_out_b"]
+    h_s = W["state_w"] @ state + W["state_b"]
+    return np.concatenate([h_s[None, :], h_a], axis=0)
+
+
+def pi0_velocity(W, x, state, t, k_pref, v_pref, lv, cfg, trace=None):
+    """v_t of one sample: suffix tokens -> L π0 layers -> final RMSNorm -> action_out_proj on
+    the action tokens (reading P5)."""
+    h = pi0_suffix(W, x, state, t, cfg)
+    if trace is not None:
+        trace.append(h.copy())
+    for l in range(cfg.n_layers):
+        h = pi0_layer(h, W, l, k_pref[l], v_pref[l], lv, cfg)
+        if trace is not None:
+            trace.append(h.copy())
+    n = rms_normalize(h, cfg.rms_eps) * (1.0 + W["final_ln"])
+    return n[1:] @ W["action_out_w"].T + W["action_out_b"]
+
+
+def pi0_sample_actions(weights, cfg, noise, state, kv_k, kv_v, valid_len, trace_step=None):
+    """The π0 Euler loop: x_{t+dt} = x_t + dt * v_t, dt = -1/S, t_k = 1 - k/S (R12).
+
+    noise [B, C, A]; state [B, A]; kv_k, kv_v [L, B, P, hd]; valid_len [B].  Returns actions
+    [B, C, A] and, if trace_step is given, the hidden states [L+1, B, C+1, D] of that step.
+    """
+    W = _as_weights(weights)
+    S = cfg.n_steps
+    x = np.array(noise, dtype=F64)
+    st = np.asarray(state, dtype=F64)
+    B, C = x.shape[0], x.shape[1]
+    tr = None if trace_step is None else np.zeros((cfg.n_layers + 1, B, C + 1, cfg.width), dtype=F64)
+    kk, vv = np.asarray(kv_k), np.asarray(kv_v)
+    for k in range(S):
+        t = 1.0 - k / S
+        for b in range(B):
+            lst = [] if (trace_step is not None and k == trace_step) else None
+            v = pi0_velocity(W, x[b], st[b], t, kk[:, b].astype(F64), vv[:, b].astype(F64),
+                             int(valid_len[b]), cfg, lst)
+            x[b] = x[b] + (-1.0 / S) * v
+            if lst is not None:
+                tr[:, b] = np.stack(lst)
+    return (x, tr) if trace_step is not None else x

@@ -116,6 +116,45 @@ def expert_weight_shapes(s: ExpertShape) -> dict:
     return shapes
 
 
+def pi0_expert_weight_shapes(s: ExpertShape) -> dict:
+    """The π0 action expert: state projection, action-time MLP, plain RMSNorm weights."""
+    D, F, H, hd, A = s.width, s.mlp_dim, s.n_q_heads, s.head_dim, s.action_dim
+    kvd = s.n_kv_heads * hd
+    shapes = {
+        "action_in_w": (D, A), "action_in_b": (D,),
+        "action_out_w": (A, D), "action_out_b": (A,),
+        "state_w": (D, A), "state_b": (D,),
+        "action_time_in_w": (D, 2 * D), "action_time_in_b": (D,),
+        "action_time_out_w": (D, D), "action_time_out_b": (D,),
+        "final_ln": (D,),
+    }
+    for l in range(s.n_layers):
+        shapes.update({
+            f"l{l}.wq": (H * hd, D), f"l{l}.wk": (kvd, D), f"l{l}.wv": (kvd, D),
+            f"l{l}.wo": (D, H * hd),
+            f"l{l}.wg": (F, D), f"l{l}.wu": (F, D), f"l{l}.wd": (D, F),
+            f"l{l}.ln1": (D,), f"l{l}.ln2": (D,),
+        })
+    return shapes
+
+
+def pi0_expert_weights(s: ExpertShape, std: float = 0.02, bias_std: float = 0.0,
+                       tag: str = "pi0") -> dict:
+    """bf16 bit patterns of every π0 expert tensor; RMSNorm weights w (scale 1 + w) N(0, std^2)."""
+    out = {}
+    for name, shape in pi0_expert_weight_shapes(s).items():
+        if _is_bias(name) and bias_std <= 0:
+            out[name] = np.zeros(shape, dtype=np.uint16)
+        else:
+            out[name] = gen.normal_bf16(f"{tag}/{name}", shape, bias_std if _is_bias(name) else std)
+    return out
+
+
+def state(w: Workload, tag: str = "state") -> np.ndarray:
+    """π0 robot state, float32 N(0, 1) [B][action_dim]."""
+    return gen.normal(f"{tag}/{w.batch}", (w.batch, w.expert.action_dim), 1.0)
+
+
 def prefill_weight_shapes(s: PrefillShape) -> dict:
     D, F, H, hd = s.width, s.mlp_dim, s.n_q_heads, s.head_dim
     kvd = s.n_kv_heads * hd
@@ -194,5 +233,6 @@ def as_f32(bits_dict: dict) -> dict:
 
 
 __all__ = ["ExpertShape", "PrefillShape", "Workload", "workload", "expert_weights",
+           "pi0_expert_weight_shapes", "pi0_expert_weights", "state",
            "prefill_weights", "kv_cache", "noise", "prefill_inputs", "as_f32",
            "expert_weight_shapes", "prefill_weight_shapes", "replace", "field"]

@@ -492,3 +492,178 @@ def test_golden_regression_of_the_oracle():
     stored = json.load(open(os.path.join(here, "tiny_expert_actions.json")))
     expect = np.array([float.fromhex(x) for x in stored["actions"]]).reshape(stored["shape"])
     np.testing.assert_allclose(mg.compute(), expect, rtol=1e-12, atol=1e-12)
+
+
+# The same planted mistakes at full size (18 layers, width 1024, 1-view: chunk 50, 280 of 288
+# prefix tokens valid) with PLAIN N(0, 0.02) weights, caught by the per-layer check the GPU
+# tests apply (every layer's hidden state and update within relative L2 1e-2).  On plain
+# weights a check of the final actions alone misses several of them, because each layer's
+# update is small next to h; the per-layer updates are not.  Step 0 of the loop is traced
+# (the trace of step 0 depends only on t_0 = 1, so one Euler step suffices).
+
+@pytest.fixture(scope="module")
+def plain_full_size():
+    from dataclasses import replace
+    w = WL.workload(2)
+    one = replace(w.expert, n_steps=1)
+    Wt = M.Weights(WL.as_f32(WL.expert_weights(w.expert)))
+    k, v, lv = WL.kv_cache(w)
+    kf, vf = gen.bf16_to_f32(k), gen.bf16_to_f32(v)
+    x0 = WL.noise(w)
+    _, tr = M.sample_actions(Wt, one, x0, kf, vf, lv, trace_step=0)
+    return one, Wt, kf, vf, lv, x0, tr
+
+
+def _fails_per_layer(tr, rtr):
+    return any(rel_l2(tr[i], rtr[i]) > H_REL_L2 for i in range(tr.shape[0])) or any(
+        rel_l2(tr[i] - tr[i - 1], rtr[i] - rtr[i - 1]) > H_REL_L2 for i in range(1, tr.shape[0]))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS) + ["valid_len_plus_one"])
+def test_mutants_fail_the_per_layer_check_at_full_size(plain_full_size, monkeypatch, name):
+    one, Wt, kf, vf, lv, x0, rtr = plain_full_size
+    if name == "valid_len_plus_one":
+        _, tr = M.sample_actions(Wt, one, x0, kf, vf, lv + 1, trace_step=0)
+    else:
+        MUTANTS[name](monkeypatch)
+        _, tr = M.sample_actions(Wt, one, x0, kf, vf, lv, trace_step=0)
+    assert _fails_per_layer(tr, rtr), name
+
+
+# ---------------------------------------------------------------------------------------
+# the π0 suffix variant (readings P1-P5 in oracle/model.py)
+
+def rand_pi0_weights(cfg, std=0.3, bias_std=0.1, rng=RNG):
+    shapes = WL.pi0_expert_weight_shapes(cfg)
+    return {k: rng.normal(0, bias_std if k.endswith("_b") else std, size=s) for k, s in shapes.items()}
+
+
+def _torch_pi0_sample_actions(W, cfg, noise, state, kk, vv, lv):
+    """An independent torch fp64 formulation of the π0 loop: F.linear / F.rms_norm / SDPA with a
+    boolean mask / complex-rotation RoPE; the suffix built as one [state ; actions] tensor."""
+    T = {k: torch.from_numpy(np.asarray(v, dtype=np.float64)) for k, v in W.items()}
+    D, H, hd = cfg.width, cfg.n_q_heads, cfg.head_dim
+    x = torch.from_numpy(noise.astype(np.float64)).clone()
+    st = torch.from_numpy(np.asarray(state, dtype=np.float64))
+    half = D // 2
+    for step in range(cfg.n_steps):
+        t = 1.0 - step / cfg.n_steps
+        per = 4e-3 * (1000.0 ** (torch.arange(half, dtype=torch.float64) / (half - 1)))
+        e = torch.cat([torch.sin(2 * math.pi * t / per), torch.cos(2 * math.pi * t / per)])
+        for b in range(x.shape[0]):
+            C = x.shape[1]
+            P = kk.shape[2]
+            a = F.linear(x[b], T["action_in_w"], T["action_in_b"])
+            at = torch.cat([a, e.expand(C, D)], dim=1)
+            ha = F.linear(F.silu(F.linear(at, T["action_time_in_w"], T["action_time_in_b"])),
+                          T["action_time_out_w"], T["action_time_out_b"])
+            h = torch.cat([F.linear(st[b], T["state_w"], T["state_b"])[None], ha], 0)
+            Tn = C + 1
+            for l in range(cfg.n_layers):
+                n = F.rms_norm(h, (D,), weight=1 + T[f"l{l}.ln1"], eps=cfg.rms_eps)
+                q = F.linear(n, T[f"l{l}.wq"]).view(Tn, H, hd).transpose(0, 1)
+                k = F.linear(n, T[f"l{l}.wk"]).view(Tn, 1, hd).transpose(0, 1)
+                v = F.linear(n, T[f"l{l}.wv"]).view(Tn, 1, hd).transpose(0, 1)
+                pos = list(range(int(lv[b]), int(lv[b]) + Tn))
+                q, k = _torch_rope(q, pos, cfg.rope_theta), _torch_rope(k, pos, cfg.rope_theta)
+                Kall = torch.cat([torch.from_numpy(kk[l, b][None].astype(np.float64)), k], 1).expand(H, P + Tn, hd)
+                Vall = torch.cat([torch.from_numpy(vv[l, b][None].astype(np.float64)), v], 1).expand(H, P + Tn, hd)
+                allowed = torch.cat([torch.arange(P) < int(lv[b]), torch.ones(Tn, dtype=torch.bool)])
+                o = F.scaled_dot_product_attention(q, Kall, Vall, attn_mask=allowed[None, :].expand(Tn, P + Tn))
+                h = h + F.linear(o.transpose(0, 1).reshape(Tn, H * hd), T[f"l{l}.wo"])
+                n = F.rms_norm(h, (D,), weight=1 + T[f"l{l}.ln2"], eps=cfg.rms_eps)
+                h = h + F.linear(F.gelu(F.linear(n, T[f"l{l}.wg"]), approximate="tanh") * F.linear(n, T[f"l{l}.wu"]),
+                                 T[f"l{l}.wd"])
+            n = F.rms_norm(h, (D,), weight=1 + T["final_ln"], eps=cfg.rms_eps)
+            x[b] = x[b] - 0.1 * F.linear(n[1:], T["action_out_w"], T["action_out_b"])
+    return x.numpy()
+
+
+def _pi0_inputs(cfg, B=2, C=3, P=6, lv=(4, 6)):
+    noise, kk, vv, lvs = _tiny_inputs(cfg, B=B, C=C, P=P, lv=lv)
+    return noise, RNG.normal(size=(B, cfg.action_dim)), kk, vv, lvs
+
+
+def test_pi0_loop_matches_independent_torch_formulation():
+    cfg = tiny_expert()
+    W = rand_pi0_weights(cfg)
+    noise, state, kk, vv, lv = _pi0_inputs(cfg)
+    out = M.pi0_sample_actions(W, cfg, noise, state, kk, vv, lv)
+    ref = _torch_pi0_sample_actions(W, cfg, noise, state, kk, vv, lv)
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-10)
+    assert rel_l2(out, noise) > 0.05
+
+
+def test_pi0_action_time_fold_and_table():
+    """The folding the library applies at create time: Linear_in([W_a x + b_a ; e(t)]) =
+    (W_in[:, :D] W_a) x + (W_in[:, :D] b_a + W_in[:, D:] e(t) + b_in), one table row per t."""
+    cfg = tiny_expert()
+    W = rand_pi0_weights(cfg)
+    D = cfg.width
+    Wi, bi = W["action_time_in_w"], W["action_time_in_b"]
+    x = RNG.normal(size=(5, cfg.action_dim))
+    fold = Wi[:, :D] @ W["action_in_w"]
+    for k in range(cfg.n_steps):
+        t = 1.0 - k / cfg.n_steps
+        e = M.sinusoidal_time_embedding(t, D)
+        direct = np.concatenate([x @ W["action_in_w"].T + W["action_in_b"], np.broadcast_to(e, (5, D))], 1) @ Wi.T + bi
+        table = Wi[:, :D] @ W["action_in_b"] + Wi[:, D:] @ e + bi
+        np.testing.assert_allclose(x @ fold.T + table, direct, rtol=1e-12, atol=1e-12)
+
+
+def test_pi0_euler_closed_form_and_state_only_through_attention():
+    cfg = tiny_expert()
+    W = rand_pi0_weights(cfg)
+    noise, state, kk, vv, lv = _pi0_inputs(cfg)
+    beta = RNG.normal(size=cfg.action_dim)
+    Z = dict(W, action_out_w=np.zeros_like(W["action_out_w"]), action_out_b=beta)
+    np.testing.assert_allclose(M.pi0_sample_actions(Z, cfg, noise, state, kk, vv, lv), noise - beta,
+                               rtol=0, atol=1e-12)
+    # the state token reaches the actions only through attention: with every o_proj zero, the
+    # actions ignore the state (and the prefix); with them, they do not
+    Wz = dict(W)
+    for l in range(cfg.n_layers):
+        Wz[f"l{l}.wo"] = np.zeros_like(W[f"l{l}.wo"])
+    a = M.pi0_sample_actions(Wz, cfg, noise, state, kk, vv, lv)
+    b = M.pi0_sample_actions(Wz, cfg, noise, state + 1.0, kk * -1.0, vv, lv)
+    np.testing.assert_array_equal(a, b)
+    c = M.pi0_sample_actions(W, cfg, noise, state, kk, vv, lv)
+    d = M.pi0_sample_actions(W, cfg, noise, state + 1.0, kk, vv, lv)
+    assert np.abs(c - d).max() > 1e-3
+
+
+def test_pi0_suffix_positions_and_state_row():
+    """The suffix is [state ; actions]: the trace has C + 1 rows per step and its first row
+    entering layer 0 is the state projection W_s state + b_s (reading P1)."""
+    cfg = tiny_expert()
+    W = M.Weights(rand_pi0_weights(cfg))
+    noise, state, kk, vv, lv = _pi0_inputs(cfg, B=1, lv=(4,))
+    _, tr = M.pi0_sample_actions(W, cfg, noise, state, kk, vv, lv, trace_step=0)
+    np.testing.assert_allclose(tr[0, 0, 0], W["state_w"] @ state[0] + W["state_b"], rtol=1e-13, atol=1e-13)
+    assert tr.shape == (cfg.n_layers + 1, 1, noise.shape[1] + 1, cfg.width)
+
+
+PI0_MUTANTS = {
+    "no_state_token": lambda mp: mp.setattr(
+        M, "pi0_suffix", (lambda f: lambda W, x, s, t, cfg: np.concatenate(
+            [np.zeros((1, cfg.width)), f(W, x, s, t, cfg)[1:]], 0))(M.pi0_suffix)),
+    "time_embedding_dropped": lambda mp: mp.setattr(
+        M, "sinusoidal_time_embedding", lambda t, dim, **k: np.zeros(dim)),
+    "no_rope": lambda mp: mp.setattr(M, "rope", lambda x, pos, theta: x),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PI0_MUTANTS))
+def test_pi0_mutants_fail_parity(monkeypatch, name):
+    """On the full-width 2-layer π0 expert with N(0, 0.02) weights, each planted mistake moves
+    the actions or a layer's update beyond the parity tolerance."""
+    from dataclasses import replace
+    w = WL.workload(1)
+    Wt = M.Weights(WL.as_f32(WL.pi0_expert_weights(w.expert, bias_std=0.02)))
+    k, v, lv = WL.kv_cache(w)
+    kf, vf = gen.bf16_to_f32(k), gen.bf16_to_f32(v)
+    x0, st = WL.noise(w), WL.state(w)
+    ref, rtr = M.pi0_sample_actions(Wt, w.expert, x0, st, kf, vf, lv, trace_step=0)
+    PI0_MUTANTS[name](monkeypatch)
+    out, tr = M.pi0_sample_actions(Wt, w.expert, x0, st, kf, vf, lv, trace_step=0)
+    assert _fails_parity(out, tr, ref, rtr), name
