@@ -40,10 +40,11 @@ def parse():
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--engine", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--workload", default="2-view", choices=["2-view", "1-view", "3-view", "e2e", "stream"],
+    p.add_argument("--workload", default="2-view", choices=["2-view", "1-view", "3-view", "e2e", "stream", "pi0"],
                    help="2-view (the headline line), 1-view, 3-view (with --batch), e2e: prefill of the "
                         "544-token prefix, then the denoise loop; stream: frames of e2e back to back, the "
-                        "prefill of frame n+1 overlapping the denoise of frame n (layered engine)")
+                        "prefill of frame n+1 overlapping the denoise of frame n (layered engine); pi0: the "
+                        "2-view workload on the pi0 suffix variant (state token, action-time MLP)")
     return p.parse_args()
 
 
@@ -88,6 +89,24 @@ def prefill_algorithmic(wl):
     flops = (s.n_layers - 1) * (2 * T * full + sum(4 * H * l * l * hd for l in wl.valid_lens)) + 2 * T * kv_only
     bytes_ = ((s.n_layers - 1) * full + kv_only) * 2 + s.n_layers * wl.batch * wl.prefix_cap * kvd * 2 * 2
     return bytes_, flops
+
+
+def pi0_algorithmic(wl):
+    """Bytes and FLOPs of one 10-step pi0 loop: the 18 layers' weights, the folded action-time
+    MLP (fp32 W_fold [1024][32] and its output linear), state and action projections, the
+    valid prefix KV, the norm tables and the suffix K/V of C + 1 tokens."""
+    s = wl.expert
+    L, D, F, H, hd, A, S = s.n_layers, s.width, s.mlp_dim, s.n_q_heads, s.head_dim, s.action_dim, s.n_steps
+    per_layer_params = (H * hd + 2 * hd) * D + D * H * hd + 2 * F * D + D * F
+    T = wl.chunk + 1
+    M = wl.batch * T
+    bf16_params = L * per_layer_params + D * D + 2 * D * A      # layers, action-time out, state + action out
+    lv = sum(wl.valid_lens)
+    bytes_step = (bf16_params * 2 + D * A * 4 + D * 4 + L * lv * hd * 2 * 2 + L * 2 * D * 4
+                  + L * M * hd * 2 * 2 * 2)
+    attn = sum(4 * H * T * (l + T) * hd for l in wl.valid_lens) * L
+    flops_step = 2 * M * (L * per_layer_params + D * D) + 2 * wl.batch * wl.chunk * (D * A * 2) + attn
+    return bytes_step * S, flops_step * S
 
 
 def algorithmic(wl):
@@ -306,6 +325,8 @@ def run_ours(args, rank, world, local_rank):
         return run_e2e(args, rank, world, local_rank, wl)
     if args.workload == "stream":
         return run_stream(args, rank, world, local_rank, wl)
+    if args.workload == "pi0":
+        return run_pi0(args, rank, world, local_rank, wl)
     bits = WL.expert_weights(wl.expert)
     dw = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev) for k, v in bits.items()}
     cfg = R.make_config(n_layers=wl.expert.n_layers, chunk=wl.chunk, max_prefix=wl.prefix_cap,
@@ -418,6 +439,109 @@ def run_ours(args, rank, world, local_rank):
         line["cpu_baseline"] = {"value": round(statistics.mean(times), 1), "unit": "ms", "cores": cpu_threads(),
                                 "kind": "oracle",
                                 "sample": f"3 full {wl.expert.n_steps}-step loops of the same workload (fp64 oracle)"}
+    print(json.dumps(line), flush=True)
+
+
+def run_pi0(args, rank, world, local_rank, wl):
+    """The 2-view workload on the pi0 suffix variant: the suffix is [state token ; 63 action
+    tokens], the action tokens come from the folded action-time MLP, plain RMSNorm, ungated
+    residuals (layered engine).  e2e: pinned host noise, state and cache copied in, the call,
+    the actions copied out, all inside the timed region."""
+    import torch
+
+    import flow_matching_action_expert_b200 as R
+    from synth import workloads as WL
+
+    dev = torch.device("cuda", local_rank)
+    bits = WL.pi0_expert_weights(wl.expert, bias_std=0.02)
+    dw = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev) for k, v in bits.items()}
+    cfg = R.make_config(n_layers=wl.expert.n_layers, chunk=wl.chunk, max_prefix=wl.prefix_cap,
+                        max_batch=wl.batch, engine=args.engine, variant=R.VARIANT_PI0)
+    ctx = R.rtvla_create(dw, cfg)
+    del dw
+    kb, vb, valid = WL.kv_cache(wl)
+    noise_np, state_np = WL.noise(wl), WL.state(wl)
+    k = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).to(dev)
+    v = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16).to(dev)
+    vl = torch.from_numpy(valid).to(dev)
+    noise = torch.from_numpy(noise_np).to(dev)
+    state = torch.from_numpy(state_np).to(dev)
+    out = torch.empty_like(noise)
+    kv = R.make_kv(k, v, vl, wl.batch, wl.prefix_cap)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def call():
+        R.rtvla_sample_actions_pi0(ctx, noise, state, kv, out, stream)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    st = R.rtvla_sync_status(ctx, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {R.STATUS[st]}")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    per = [a.elapsed_time(b) for a, b in ev]
+    ms = reduce_max([statistics.mean(per)], dev)[0]
+    kernels = R.rtvla_kernels_per_call(ctx, wl.batch)
+    # end to end: pinned host inputs in, the call, the actions out
+    hk = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hl, hn = torch.from_numpy(valid).pin_memory(), torch.from_numpy(noise_np).pin_memory()
+    hs, ho = torch.from_numpy(state_np).pin_memory(), torch.empty_like(hn).pin_memory()
+    e2e = []
+    for i in range(args.steps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for d, h in ((noise, hn), (state, hs), (k, hk), (v, hv), (vl, hl)):
+            d.copy_(h, non_blocking=True)
+        call()
+        ho.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= 2:
+            e2e.append(e0.elapsed_time(e1))
+    e2e_ms = reduce_max([statistics.mean(e2e)], dev)[0]
+    st = R.rtvla_sync_status(ctx, stream)
+    R.rtvla_destroy(ctx)
+    if st != 0:
+        raise RuntimeError(f"device status {R.STATUS[st]}")
+    if rank != 0:
+        return
+    hbm, bf16_pk, bf16_sus, src = peaks()
+    b_loop, f_loop = pi0_algorithmic(wl)
+    t_mem, t_tc = b_loop / (hbm * 1e9), f_loop / (bf16_sus * 1e12)
+    gbs = b_loop / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "pi0 10-step denoise latency ms (2-view, chunk 63 + state token)", "value": round(ms, 4),
+        "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) bf16 weights and biases, N(0,1) KV, noise, state)",
+        "config": dict(workload_config(wl, world), workload="pi0 " + wl.name, suffix_tokens=wl.chunk + 1),
+        "engine": "layered", "l2": "flushed by a 256 MiB write between timed loops",
+        "roofline": {"bound": "hbm" if t_mem >= t_tc else "tensor",
+                     "kernel": "rtvla_sample_actions_pi0 (one graph replay)",
+                     "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                     "traffic": None, "peak_source": src, "algorithmic_bytes_per_launch": int(b_loop),
+                     "algorithmic_flops_per_launch": int(f_loop), "roofline_ms": round(max(t_mem, t_tc) * 1e3, 4)},
+        "e2e": {"value": round(e2e_ms, 4), "unit": "ms",
+                "h2d_bytes_per_step": int(hn.numel() * 4 + hs.numel() * 4 + hk.numel() * 2 * 2 + hl.numel() * 4),
+                "d2h_bytes_per_step": int(ho.numel() * 4)},
+        "gpu_launches": int(kernels * args.steps) if kernels > 0 else None, "kernels_per_step": kernels,
+        "clocks": clk.summary(),
+    }
     print(json.dumps(line), flush=True)
 
 

@@ -14,11 +14,12 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "librtvla.so")
 
 ENGINE_AUTO, ENGINE_LAYERED, ENGINE_PERSISTENT = 0, 1, 2
+VARIANT_PI05, VARIANT_PI0 = 0, 1
 
 STATUS = {
     0: "RTVLA_OK", 1: "RTVLA_ERR_INVALID_ARG", 2: "RTVLA_ERR_SHAPE", 3: "RTVLA_ERR_MASK_NOT_PREFIX",
     4: "RTVLA_ERR_OOM", 5: "RTVLA_ERR_CUDA", 6: "RTVLA_ERR_DEVICE_TIMEOUT", 7: "RTVLA_ERR_UNSUPPORTED",
-    8: "RTVLA_ERR_DEVICE_BOUNDS",
+    8: "RTVLA_ERR_DEVICE_BOUNDS", 9: "RTVLA_ERR_GUARD_OVERWRITE",
 }
 
 # the symbols include/rtvla.h declares
@@ -26,7 +27,8 @@ EXPORTS = (
     "rtvla_create", "rtvla_kv_bytes", "rtvla_prefill", "rtvla_sample_actions", "rtvla_sample_actions_host",
     "rtvla_sample_actions_host_static",
     "rtvla_sync_status", "rtvla_debug_trace", "rtvla_kernels_per_call", "rtvla_set_engine",
-    "rtvla_set_wait_timeout_us", "rtvla_destroy", "rtvla_status_string",
+    "rtvla_set_wait_timeout_us", "rtvla_destroy", "rtvla_status_string", "rtvla_debug_plant_guard_fault",
+    "rtvla_sample_actions_pi0", "rtvla_debug_trace_pi0",
 )
 
 
@@ -41,7 +43,7 @@ class RtvlaConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "n_layers", "width", "mlp_dim", "n_q_heads", "n_kv_heads", "head_dim", "action_dim", "chunk",
         "n_steps", "max_prefix", "max_batch", "final_norm", "has_prefill", "pf_width", "pf_mlp_dim",
-        "engine")] + [("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float)]
+        "engine")] + [("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("variant", ctypes.c_int)]
 
 
 _P = ctypes.c_void_p
@@ -52,11 +54,14 @@ _SINGLE = ("action_in_w", "action_in_b", "action_out_w", "action_out_b", "time_i
 _LAYER = ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "ada_attn_w", "ada_attn_b", "ada_ffn_w", "ada_ffn_b")
 _FINAL = ("ada_final_w", "ada_final_b")
 _PF = ("pf_ln1", "pf_wq", "pf_wk", "pf_wv", "pf_wo", "pf_ln2", "pf_wg", "pf_wu", "pf_wd")
+_PI0 = ("state_w", "state_b", "action_time_in_w", "action_time_in_b", "action_time_out_w", "action_time_out_b")
+_PI0_LAYER = ("ln1", "ln2")
 
 
 class RtvlaWeights(ctypes.Structure):
     _fields_ = ([(n, _P) for n in _SINGLE] + [(n, _PP) for n in _LAYER] + [(n, _P) for n in _FINAL]
-                + [(n, _PP) for n in _PF])
+                + [(n, _PP) for n in _PF] + [(n, _P) for n in _PI0] + [(n, _PP) for n in _PI0_LAYER]
+                + [("final_ln", _P)])
 
 
 class RtvlaKV(ctypes.Structure):
@@ -80,11 +85,14 @@ def _lib():
         lib.rtvla_sample_actions.argtypes = [_P, _P, ctypes.POINTER(RtvlaKV), _P, _P]
         lib.rtvla_sample_actions_host.argtypes = [_P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P]
         lib.rtvla_sample_actions_host_static.argtypes = [_P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P]
+        lib.rtvla_sample_actions_pi0.argtypes = [_P, _P, _P, ctypes.POINTER(RtvlaKV), _P, _P]
+        lib.rtvla_debug_trace_pi0.argtypes = [_P, _P, _P, ctypes.POINTER(RtvlaKV), ctypes.c_int, _P, _P]
         lib.rtvla_sync_status.argtypes = [_P, _P]
         lib.rtvla_debug_trace.argtypes = [_P, _P, ctypes.POINTER(RtvlaKV), ctypes.c_int, _P, _P]
         lib.rtvla_kernels_per_call.argtypes = [_P, ctypes.c_int]
         lib.rtvla_set_engine.argtypes = [_P, ctypes.c_int]
         lib.rtvla_set_wait_timeout_us.argtypes = [_P, ctypes.c_longlong]
+        lib.rtvla_debug_plant_guard_fault.argtypes = [_P]
         lib.rtvla_destroy.argtypes = [_P]
         lib.rtvla_destroy.restype = None
         lib.rtvla_status_string.argtypes = [ctypes.c_int]
@@ -124,13 +132,14 @@ def _stream(s) -> int:
 
 
 def make_config(n_layers=18, chunk=63, max_prefix=512, max_batch=1, n_steps=10, final_norm=True,
-                has_prefill=False, engine=ENGINE_AUTO, rms_eps=1e-6, rope_theta=10000.0) -> RtvlaConfig:
-    """rtvla_config for the π0.5 shapes (width 1024 / MLP 4096 / 8 x 256 heads / action 32)."""
+                has_prefill=False, engine=ENGINE_AUTO, rms_eps=1e-6, rope_theta=10000.0,
+                variant=VARIANT_PI05) -> RtvlaConfig:
+    """rtvla_config for the π0.5 / π0 shapes (width 1024 / MLP 4096 / 8 x 256 heads / action 32)."""
     return RtvlaConfig(n_layers=n_layers, width=1024, mlp_dim=4096, n_q_heads=8, n_kv_heads=1, head_dim=256,
                        action_dim=32, chunk=chunk, n_steps=n_steps, max_prefix=max_prefix,
                        max_batch=max_batch, final_norm=int(bool(final_norm)),
                        has_prefill=int(bool(has_prefill)), pf_width=2048, pf_mlp_dim=16384,
-                       engine=engine, rms_eps=rms_eps, rope_theta=rope_theta)
+                       engine=engine, rms_eps=rms_eps, rope_theta=rope_theta, variant=variant)
 
 
 def make_weights(w: dict, n_layers: int):
@@ -140,9 +149,11 @@ def make_weights(w: dict, n_layers: int):
     """
     keep = []
     ws = RtvlaWeights()
-    for n in _SINGLE + _FINAL:
+    for n in _SINGLE + _FINAL + _PI0 + ("final_ln",):
         setattr(ws, n, _ptr(w.get(n)))
-    for n in _LAYER:
+    for n in _LAYER + _PI0_LAYER:
+        if not any(f"l{l}.{n}" in w for l in range(n_layers)):
+            continue
         arr = (_P * n_layers)(*[_ptr(w.get(f"l{l}.{n}")) for l in range(n_layers)])
         keep.append(arr)
         setattr(ws, n, ctypes.cast(arr, _PP))
@@ -199,6 +210,16 @@ def rtvla_sample_actions_host_static(ctx: int, noise, kv_k, kv_v, valid_len, bat
            "rtvla_sample_actions_host_static")
 
 
+def rtvla_sample_actions_pi0(ctx: int, noise, state, kv: RtvlaKV, actions_out, stream=None):
+    _check(_lib().rtvla_sample_actions_pi0(ctx, _ptr(noise), _ptr(state), ctypes.byref(kv), _ptr(actions_out),
+                                           _stream(stream)), "rtvla_sample_actions_pi0")
+
+
+def rtvla_debug_trace_pi0(ctx: int, noise, state, kv: RtvlaKV, step: int, h_layers, stream=None):
+    _check(_lib().rtvla_debug_trace_pi0(ctx, _ptr(noise), _ptr(state), ctypes.byref(kv), step, _ptr(h_layers),
+                                        _stream(stream)), "rtvla_debug_trace_pi0")
+
+
 def rtvla_sync_status(ctx: int, stream=None) -> int:
     """Returns the device status code (0 = ok); does not raise."""
     return _lib().rtvla_sync_status(ctx, _stream(stream))
@@ -219,6 +240,10 @@ def rtvla_set_engine(ctx: int, engine: int):
 
 def rtvla_set_wait_timeout_us(ctx: int, us: int):
     _check(_lib().rtvla_set_wait_timeout_us(ctx, us), "rtvla_set_wait_timeout_us")
+
+
+def rtvla_debug_plant_guard_fault(ctx: int):
+    _check(_lib().rtvla_debug_plant_guard_fault(ctx), "rtvla_debug_plant_guard_fault")
 
 
 def rtvla_destroy(ctx: int):

@@ -14,7 +14,7 @@ typedef __nv_bfloat16 bf16;
 
 // ---------------------------------------------------------------------------------------
 // device error word (read and cleared by rtvla_sync_status)
-enum : int { DEVERR_TIMEOUT = 1, DEVERR_BOUNDS = 2, DEVERR_MASK = 4 };
+enum : int { DEVERR_TIMEOUT = 1, DEVERR_BOUNDS = 2, DEVERR_MASK = 4, DEVERR_GUARD = 8 };
 
 struct DevCtl {
   int err;                       // OR of DEVERR_*
@@ -38,6 +38,7 @@ struct CallArgs {
   bf16 *kvo_v;
   int *valid_out;
   int pf_len;           // prefill tokens per sample
+  const float *state;   // π0: robot state [batch][32]
   // persistent engine: grid-barrier arrival counters, 8 of them 128 bytes apart (all 0 in every
   // copy from the host)
   alignas(128) unsigned int bar_count[8 * 32];
@@ -216,6 +217,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
                "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+// 1-D bulk copy shared -> global (16-byte aligned addresses, size a multiple of 16), in the
+// current bulk async-group
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+               "r"(bytes)
                : "memory");
 }
 // wait until at most N committed bulk groups are still reading their shared-memory source

@@ -69,7 +69,9 @@ cudaError_t attn_launch(const AttnParams &p, int batch, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------
 // element-wise / row kernels
-cudaError_t launch_init_x(const CallArgs *ca, float *x, int n, cudaStream_t st);
+cudaError_t launch_init_x(const CallArgs *ca, float *x, int n, int Ct, int first, cudaStream_t st);
+cudaError_t launch_pi0_in(const float *x, const float *w_fold, const float *c_k, const bf16 *w_st, const float *b_st,
+                          const float *b_ato, const CallArgs *ca, float *h, bf16 *op, int M, int Ct, cudaStream_t st);
 cudaError_t launch_action_in(const float *x, const bf16 *w_in, const float *b_in, float *h, int M,
                              cudaStream_t st);
 cudaError_t launch_adanorm(const float *h, const float *s1p, bf16 *op, float *r, int M, float eps,
@@ -81,7 +83,7 @@ cudaError_t launch_gelu_mul(float *acc, const float *r, const float *bias, bf16 
                             cudaStream_t st);
 cudaError_t launch_final(const float *h, const float *s1p, const float *shift, const float *w_out,
                          const float *b_out, float *x, int M, int final_norm, float eps, const CallArgs *ca,
-                         int write_actions, cudaStream_t st);
+                         int write_actions, int Ct, int first, cudaStream_t st);
 // prefix pass
 cudaError_t launch_pf_mask(const CallArgs *ca, int B, int P, DevCtl *ctl, cudaStream_t st);
 cudaError_t launch_pf_embed(const CallArgs *ca, float *x, int M, int Dp, cudaStream_t st);
@@ -95,5 +97,16 @@ cudaError_t launch_rows_dot_f64(const bf16 *W, int R, int Kd, const double *vecs
                                 double *out, cudaStream_t st);
 cudaError_t launch_fold_cols(const bf16 *W, int R, int Kd, const bf16 *gamma, bf16 *out, cudaStream_t st);
 cudaError_t launch_scale_to_f32(const bf16 *w, int n, double s, float *out, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------
+// checked mode: guard bands of GUARD_BYTES filled with GUARD_FILL before and after every
+// library buffer; the checker flags (DEVERR_GUARD) and refills every band that changed
+constexpr int GUARD_BYTES = 4096;
+constexpr unsigned char GUARD_FILL = 0xA5;
+struct GuardRegion {
+  unsigned char *base;       // front band at [base, base + GUARD_BYTES)
+  unsigned long long bytes;  // buffer bytes (a multiple of 256); back band right after them
+};
+cudaError_t launch_check_guards(const GuardRegion *regions, int n, DevCtl *ctl, cudaStream_t st);
 
 }  // namespace rtvla

@@ -33,6 +33,10 @@ struct PersistParams {
   // environment variable RTVLA_PHASE_STAMPS names the file rtvla_destroy writes them to
   unsigned long long *stamps;
   int max_phases;
+  // optional per-layer trace: at step trace_step the kernel writes h before layer 0 and after
+  // every layer to trace, f32 [L + 1][C][1024]; null in normal calls
+  float *trace;
+  int trace_step;
 };
 
 int persistent_smem_bytes();

@@ -26,10 +26,54 @@ __device__ __forceinline__ float block_sum_256(float v, float *red) {
 }
 }  // namespace
 
-// x = noise (copy through the call's argument block)
-__global__ void k_init_x(const CallArgs *ca, float *x, int n) {
+// x = noise (copy through the call's argument block).  The expert runs Ct token rows per
+// sample; the first `first` of them (the π0 state token) carry no action and get x = 0.
+__global__ void k_init_x(const CallArgs *ca, float *x, int n, int Ct, int first) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) x[i] = ca->noise[i];
+  if (i >= n) return;
+  const int m = i >> 5, a = i & 31, b = m / Ct, j = m % Ct;
+  x[i] = j < first ? 0.f : ca->noise[((size_t)b * (Ct - first) + (j - first)) * 32 + a];
+}
+
+// π0 suffix rows of one step ("Running VLAs at Real-time Speed" summary, "How": the two
+// linears of the action time encoder folded, the step's time rows tabulated before SiLU).
+// Row m of sample b = m / Ct: the state token (j = 0): h = W_s state_b + b_s and a zero GEMM
+// operand; an action token: operand bf16(SiLU(W_fold x + c_k)) and h = b_out of the
+// action-time MLP, to which the following GEMM adds operand @ W_out^T.
+__global__ void __launch_bounds__(256) k_pi0_in(const float *x, const float *w_fold, const float *c_k,
+                                                 const bf16 *w_st, const float *b_st, const float *b_ato,
+                                                 const CallArgs *ca, float *h, bf16 *op, int Ct) {
+  __shared__ float xs[32];
+  const int m = blockIdx.x, b = m / Ct, j = m % Ct;
+  if (threadIdx.x < 32) xs[threadIdx.x] = j == 0 ? ca->state[b * 32 + threadIdx.x] : x[m * 32 + threadIdx.x];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int n = threadIdx.x + 256 * k;
+    if (j == 0) {
+      const uint4 *wr = reinterpret_cast<const uint4 *>(w_st + n * 32);
+      float acc = b_st[n];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = wr[q];
+        const bf16 *e = reinterpret_cast<const bf16 *>(&v);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc += bf2f(e[t]) * xs[q * 8 + t];
+      }
+      h[(size_t)m * 1024 + n] = acc;
+      op[(size_t)m * 1024 + n] = f2bf(0.f);
+    } else {
+      const float4 *wr = reinterpret_cast<const float4 *>(w_fold + n * 32);
+      float acc = c_k[n];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 v = wr[q];
+        acc += v.x * xs[4 * q] + v.y * xs[4 * q + 1] + v.z * xs[4 * q + 2] + v.w * xs[4 * q + 3];
+      }
+      op[(size_t)m * 1024 + n] = f2bf(acc / (1.0f + __expf(-acc)));
+      h[(size_t)m * 1024 + n] = b_ato[n];
+    }
+  }
 }
 
 // h[m][:] = x[m][:] @ W_in^T + b_in   (action_in_proj, 32 -> 1024)
@@ -182,10 +226,12 @@ __global__ void __launch_bounds__(256) k_gelu_mul(float *__restrict__ acc, const
 // x[m] += n @ (dt W_out)^T + dt b_out.  Writes the actions when asked.
 __global__ void __launch_bounds__(256) k_final(const float *h, const float *s1p, const float *shift, const float *w_out,
                                                const float *b_out, float *x, int final_norm, float eps,
-                                               const CallArgs *ca, int write_actions) {
+                                               const CallArgs *ca, int write_actions, int Ct, int first) {
   __shared__ float n[1024];
   __shared__ float red[8];
   const int m = blockIdx.x;
+  if (m % Ct < first) return;  // the π0 state token: no action
+  const size_t arow = (size_t)(m / Ct) * (Ct - first) + (m % Ct - first);
   const float4 v = reinterpret_cast<const float4 *>(h + (size_t)m * 1024)[threadIdx.x];
   const float ss = block_sum_256(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, red);
   float4 y = v;
@@ -208,7 +254,7 @@ __global__ void __launch_bounds__(256) k_final(const float *h, const float *s1p,
     if (l == 0) {
       const float nx = x[m * 32 + a] + acc + b_out[a];
       x[m * 32 + a] = nx;
-      if (write_actions) ca->actions[m * 32 + a] = nx;
+      if (write_actions) ca->actions[arow * 32 + a] = nx;
     }
   }
 }
@@ -349,8 +395,13 @@ __global__ void k_scale_to_f32(const bf16 *w, int n, double s, float *out) {
 
 // ---------------------------------------------------------------------------------------
 // launchers
-cudaError_t launch_init_x(const CallArgs *ca, float *x, int n, cudaStream_t st) {
-  k_init_x<<<(n + 255) / 256, 256, 0, st>>>(ca, x, n);
+cudaError_t launch_init_x(const CallArgs *ca, float *x, int n, int Ct, int first, cudaStream_t st) {
+  k_init_x<<<(n + 255) / 256, 256, 0, st>>>(ca, x, n, Ct, first);
+  return cudaGetLastError();
+}
+cudaError_t launch_pi0_in(const float *x, const float *w_fold, const float *c_k, const bf16 *w_st, const float *b_st,
+                          const float *b_ato, const CallArgs *ca, float *h, bf16 *op, int M, int Ct, cudaStream_t st) {
+  k_pi0_in<<<M, 256, 0, st>>>(x, w_fold, c_k, w_st, b_st, b_ato, ca, h, op, Ct);
   return cudaGetLastError();
 }
 cudaError_t launch_action_in(const float *x, const bf16 *w_in, const float *b_in, float *h, int M, cudaStream_t st) {
@@ -373,8 +424,8 @@ cudaError_t launch_gelu_mul(float *acc, const float *r, const float *bias, bf16 
 }
 cudaError_t launch_final(const float *h, const float *s1p, const float *shift, const float *w_out, const float *b_out,
                          float *x, int M, int final_norm, float eps, const CallArgs *ca, int write_actions,
-                         cudaStream_t st) {
-  k_final<<<M, 256, 0, st>>>(h, s1p, shift, w_out, b_out, x, final_norm, eps, ca, write_actions);
+                         int Ct, int first, cudaStream_t st) {
+  k_final<<<M, 256, 0, st>>>(h, s1p, shift, w_out, b_out, x, final_norm, eps, ca, write_actions, Ct, first);
   return cudaGetLastError();
 }
 cudaError_t launch_pf_mask(const CallArgs *ca, int B, int P, DevCtl *ctl, cudaStream_t st) {
@@ -406,6 +457,39 @@ cudaError_t launch_fold_cols(const bf16 *W, int R, int Kd, const bf16 *gamma, bf
 }
 cudaError_t launch_scale_to_f32(const bf16 *w, int n, double s, float *out, cudaStream_t st) {
   k_scale_to_f32<<<(n + 255) / 256, 256, 0, st>>>(w, n, s, out);
+  return cudaGetLastError();
+}
+
+}  // namespace rtvla
+
+namespace rtvla {
+
+// One CTA per guarded buffer: both bands are compared with the fill byte 16 bytes at a time;
+// a band that changed is reported (DEVERR_GUARD, where = 700 + buffer index) and refilled.
+__global__ void k_check_guards(const GuardRegion *regions, DevCtl *ctl) {
+  const GuardRegion r = regions[blockIdx.x];
+  const uint4 fill4 = make_uint4(0xA5A5A5A5u, 0xA5A5A5A5u, 0xA5A5A5A5u, 0xA5A5A5A5u);
+  static_assert(GUARD_FILL == 0xA5, "fill word");
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  uint4 *bands[2] = {reinterpret_cast<uint4 *>(r.base),
+                     reinterpret_cast<uint4 *>(r.base + GUARD_BYTES + r.bytes)};
+  for (int b = 0; b < 2; ++b)
+    for (int i = threadIdx.x; i < GUARD_BYTES / 16; i += blockDim.x) {
+      const uint4 v = bands[b][i];
+      if (v.x != fill4.x || v.y != fill4.y || v.z != fill4.z || v.w != fill4.w) {
+        bad = 1;
+        bands[b][i] = fill4;
+      }
+    }
+  __syncthreads();
+  if (threadIdx.x == 0 && bad) set_error(ctl, DEVERR_GUARD, 700 + (int)blockIdx.x);
+}
+
+cudaError_t launch_check_guards(const GuardRegion *regions, int n, DevCtl *ctl, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  k_check_guards<<<n, 256, 0, st>>>(regions, ctl);
   return cudaGetLastError();
 }
 

@@ -37,7 +37,9 @@ constexpr int D = 1024, F = 4096, HD = 256, NQH = 8, A = 32, DP = 2048, FP = 163
 struct rtvla_ctx {
   rtvla_config cfg;
   int device = 0, sm_count = 148;
-  int L = 0, S = 0, C = 0, Bmax = 0, Pmax = 0;
+  // C: token rows per sample in the expert (the action chunk Ca, plus the state token for π0)
+  int L = 0, S = 0, C = 0, Ca = 0, Bmax = 0, Pmax = 0;
+  int variant = RTVLA_VARIANT_PI05, first = 0;  // first: rows before the action rows (π0: 1)
   int engine = RTVLA_ENGINE_AUTO;
   std::vector<void *> allocs;
   // folded / repacked expert weights (library-owned)
@@ -48,6 +50,11 @@ struct rtvla_ctx {
   float *bias_qkv = nullptr, *bias_gu = nullptr, *s1p_fin = nullptr, *shift_fin = nullptr;
   float *rope_cos = nullptr, *rope_sin = nullptr;
   int rope_rows = 0;
+  // π0: folded action-time MLP (fp32 W_fold [D][A] and the pre-SiLU table c_k [S][D]), its
+  // output linear (a GEMM weight), the state projection
+  float *pi_wfold = nullptr, *pi_ctab = nullptr, *pi_bato = nullptr, *pi_bst = nullptr;
+  bf16 *pi_wato = nullptr, *pi_wst = nullptr;
+  CUtensorMap tm_wato;
   // prefix-pass weights
   bf16 *pw_qkv = nullptr, *pw_o = nullptr, *pw_gu = nullptr, *pw_d = nullptr;
   // denoise activations
@@ -83,6 +90,12 @@ struct rtvla_ctx {
   float *st_noise = nullptr, *st_act = nullptr;
   size_t st_kv_elems = 0, st_io_elems = 0;
   int st_batch = 0;
+  // checked mode (RTVLA_CHECKED=1 at create): guard bands around every library buffer
+  bool checked = false;
+  std::vector<GuardRegion> guards;
+  GuardRegion *d_guards = nullptr;
+  // device-memory cap of this context (RTVLA_DEVICE_MEMORY_CAP bytes at create; 0 = none)
+  size_t mem_cap = 0, mem_used = 0;
 };
 
 namespace {
@@ -128,8 +141,8 @@ bool make_map_f32(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols
 // fp32 [64][cols] row-major, seen as 3-D {32 columns, 64 rows, cols / 32 column blocks} with
 // strides (row cols * 4 B, block 128 B): one box of `blocks` column blocks lands in shared
 // memory as that many consecutive 8 KB tiles [64 rows][32 columns], each with 128-byte swizzle.
-bool make_map_f32_blocks(CUtensorMap *m, const void *base, uint64_t cols, uint32_t blocks) {
-  cuuint64_t dims[3] = {32, 64, cols / 32};
+bool make_map_f32_blocks(CUtensorMap *m, const void *base, uint64_t cols, uint32_t blocks, uint64_t rows = 64) {
+  cuuint64_t dims[3] = {32, rows, cols / 32};
   cuuint64_t strides[2] = {cols * 4, 128};
   cuuint32_t box[3] = {32, 64, blocks};
   cuuint32_t es[3] = {1, 1, 1};
@@ -144,16 +157,32 @@ bool make_xmaps(XMaps *x, const void *base, uint64_t rows, uint64_t cols) {
          make_map(&x->m[2], base, rows, cols, 256);
 }
 
+// Every buffer the context owns comes from here.  A context created with a device-memory
+// cap refuses (nullptr, hence RTVLA_ERR_OOM) any allocation that would exceed it, exactly as
+// a failed cudaMalloc would be handled.  In checked mode each buffer is placed between two
+// guard bands of GUARD_BYTES filled with GUARD_FILL; rtvla_sync_status verifies them.
 template <typename T>
 T *dalloc(rtvla_ctx *c, size_t n) {
   void *p = nullptr;
   if (n == 0) n = 1;
-  if (cudaMalloc(&p, n * sizeof(T)) != cudaSuccess) {
+  const size_t bytes = (n * sizeof(T) + 255) & ~size_t(255);
+  const size_t total = c->checked ? bytes + 2 * (size_t)GUARD_BYTES : bytes;
+  if (c->mem_cap && c->mem_used + total > c->mem_cap) return nullptr;
+  if (cudaMalloc(&p, total) != cudaSuccess) {
     cudaGetLastError();
     return nullptr;
   }
   c->allocs.push_back(p);
-  return static_cast<T *>(p);
+  c->mem_used += total;
+  if (!c->checked) return static_cast<T *>(p);
+  unsigned char *b = static_cast<unsigned char *>(p);
+  if (cudaMemset(b, GUARD_FILL, GUARD_BYTES) != cudaSuccess ||
+      cudaMemset(b + GUARD_BYTES + bytes, GUARD_FILL, GUARD_BYTES) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  c->guards.push_back(GuardRegion{b, (unsigned long long)bytes});
+  return reinterpret_cast<T *>(b + GUARD_BYTES);
 }
 
 void free_all(rtvla_ctx *c) {
@@ -162,6 +191,7 @@ void free_all(rtvla_ctx *c) {
   for (auto &kv : c->graphs_pf)
     if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
   for (void *p : c->allocs) cudaFree(p);
+  if (c->d_guards) cudaFree(c->d_guards);
   if (c->st_k) cudaFree(c->st_k);
   if (c->st_v) cudaFree(c->st_v);
   if (c->st_vl) cudaFree(c->st_vl);
@@ -191,6 +221,8 @@ bool valid_cfg(const rtvla_config *c) {
   if (c->chunk < 1 || c->chunk > 256 || c->max_batch < 1 || c->max_batch > 4096) return false;
   if (c->max_prefix < 1 || c->max_prefix > 65536) return false;
   if (c->engine < 0 || c->engine > 2) return false;
+  if (c->variant != RTVLA_VARIANT_PI05 && c->variant != RTVLA_VARIANT_PI0) return false;
+  if (c->variant == RTVLA_VARIANT_PI0 && c->chunk + 1 > 256) return false;
   if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return false;
   return true;
 }
@@ -224,7 +256,7 @@ cudaError_t enqueue_denoise(rtvla_ctx *c, const CallArgs *dargs, int B, int cap,
   const float eps = c->cfg.rms_eps;
   CKR(cudaMemsetAsync(c->acc_qkv, 0, (size_t)M * 2560 * 4, st));
   CKR(cudaMemsetAsync(c->acc_gu, 0, (size_t)M * 2 * F * 4, st));
-  CKN(launch_init_x(dargs, c->x, M * A, st));
+  CKN(launch_init_x(dargs, c->x, M * A, C, c->first, st));
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
   ap.q = c->q;
@@ -240,8 +272,16 @@ cudaError_t enqueue_denoise(rtvla_ctx *c, const CallArgs *dargs, int B, int cap,
   ap.out = c->o;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
   ap.ctl = c->ctl;
+  const bool pi0 = c->variant == RTVLA_VARIANT_PI0;
   for (int k = 0; k <= last_step; ++k) {
-    CKN(launch_action_in(c->x, c->w_in, c->b_in, c->h, M, st));
+    if (pi0) {
+      // suffix rows: state projection; action tokens through the folded action-time MLP
+      CKN(launch_pi0_in(c->x, c->pi_wfold, c->pi_ctab + (size_t)k * D, c->pi_wst, c->pi_bst, c->pi_bato, dargs, c->h,
+                        c->op, M, C, st));
+      CKN(gemm_launch(c->tm_wato, 0, c->tm_op, M, D, D, c->h, c->tmo_h, D, nullptr, true, c->ctl, c->sm_count, st));
+    } else {
+      CKN(launch_action_in(c->x, c->w_in, c->b_in, c->h, M, st));
+    }
     if (trace && k == last_step)
       CKR(cudaMemcpyAsync(trace, c->h, (size_t)M * D * 4, cudaMemcpyDeviceToDevice, st));
     for (int l = 0; l < L; ++l) {
@@ -268,10 +308,10 @@ cudaError_t enqueue_denoise(rtvla_ctx *c, const CallArgs *dargs, int B, int cap,
     }
     if (!trace)
       CKN(launch_final(c->h, c->s1p_fin + (size_t)k * D, c->shift_fin + (size_t)k * D, c->w_out, c->b_out, c->x, M,
-                       c->cfg.final_norm, eps, dargs, k == S - 1 ? 1 : 0, st));
+                       c->cfg.final_norm, eps, dargs, k == S - 1 ? 1 : 0, C, c->first, st));
     else if (k < last_step)
       CKN(launch_final(c->h, c->s1p_fin + (size_t)k * D, c->shift_fin + (size_t)k * D, c->w_out, c->b_out, c->x, M,
-                       c->cfg.final_norm, eps, dargs, 0, st));
+                       c->cfg.final_norm, eps, dargs, 0, C, c->first, st));
   }
   *kernels = n;
   return cudaSuccess;
@@ -347,7 +387,8 @@ bool use_persistent(const rtvla_ctx *c, int batch) {
   return c->pers_ok && batch == 1;
 }
 
-cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, const rtvla_kv *kv, cudaStream_t st) {
+cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, const rtvla_kv *kv, cudaStream_t st,
+                              float *trace = nullptr, int trace_step = -1) {
   const int cap = kv->prefix_cap;
   c->pk_cache_k = kv->k;
   c->pk_cache_v = kv->v;
@@ -384,12 +425,12 @@ cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, const rtvla_kv *kv,
   p.rope_sin = c->rope_sin;
   p.x = c->x;
   p.h = c->h;
+  p.opart = c->pk_opart;
+  p.mlpart = c->pk_mlpart;
   p.acc_qkv = c->acc_qkv;
   p.acc_gu = c->acc_gu;
   p.ss_attn = c->ss_attn;
   p.ss_ffn = c->ss_ffn;
-  p.opart = c->pk_opart;
-  p.mlpart = c->pk_mlpart;
   p.o = c->o;
   p.qb = c->q;
   p.ks = c->ks;
@@ -397,6 +438,8 @@ cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, const rtvla_kv *kv,
   p.ctl = c->ctl;
   p.stamps = c->pk_stamps;
   p.max_phases = c->pk_max_phases;
+  p.trace = trace;
+  p.trace_step = trace_step;
   return persistent_launch(c->pmaps, p, c->sm_count, st);
 }
 
@@ -487,7 +530,77 @@ rtvla_status build_tables(rtvla_ctx *c, const rtvla_weights *w) {
     if (cudaMemcpy(u.dst, u.src->data(), u.src->size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
       return RTVLA_ERR_CUDA;
 
-  // RoPE: angle = pos * theta^(-2i/256) in fp64, rounded once to fp32
+  return RTVLA_OK;
+}
+
+// The π0 tables ("Running VLAs at Real-time Speed" summary, "How"): plain RMSNorm is the
+// AdaRMS form with scale = w, shift = 0 and gate = 1 (so the same kernels run it); the
+// action-time MLP's first linear is folded with action_in_proj, W_fold = W_in[:, :D] W_a, and
+// its 10 time rows become c_k = W_in[:, :D] b_a + W_in[:, D:] SinEmb(t_k) + b_in (fp64 on the
+// host, rounded once to fp32).
+rtvla_status build_tables_pi0(rtvla_ctx *c, const rtvla_weights *w) {
+  const int L = c->L, S = c->S;
+  std::vector<float> s1pA((size_t)S * L * D), s1pF((size_t)S * L * D), ones((size_t)S * L * D, 1.0f);
+  for (int l = 0; l < L; ++l) {
+    std::vector<double> g1 = d2h_bf16(w->ln1[l], D), g2 = d2h_bf16(w->ln2[l], D);
+    if (g1.empty() || g2.empty()) return RTVLA_ERR_CUDA;
+    for (int k = 0; k < S; ++k)
+      for (int d = 0; d < D; ++d) {
+        s1pA[((size_t)k * L + l) * D + d] = (float)(1.0 + g1[d]);
+        s1pF[((size_t)k * L + l) * D + d] = (float)(1.0 + g2[d]);
+      }
+  }
+  std::vector<double> gfin = d2h_bf16(w->final_ln, D);
+  if (gfin.empty()) return RTVLA_ERR_CUDA;
+  std::vector<float> s1pfin((size_t)S * D), shfin((size_t)S * D, 0.0f);
+  for (int k = 0; k < S; ++k)
+    for (int d = 0; d < D; ++d) s1pfin[(size_t)k * D + d] = (float)(1.0 + gfin[d]);
+  std::vector<float> zq((size_t)S * L * 2560, 0.0f), zg((size_t)S * L * 2 * F, 0.0f);
+  struct {
+    float *dst;
+    const std::vector<float> *src;
+  } up[] = {{c->s1p_attn, &s1pA}, {c->gate_attn, &ones}, {c->s1p_ffn, &s1pF}, {c->gate_ffn, &ones},
+            {c->bias_qkv, &zq},   {c->bias_gu, &zg},     {c->s1p_fin, &s1pfin}, {c->shift_fin, &shfin}};
+  for (auto &u : up)
+    if (cudaMemcpy(u.dst, u.src->data(), u.src->size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+      return RTVLA_ERR_CUDA;
+  // fold and time table
+  std::vector<double> wi = d2h_bf16(w->action_time_in_w, (size_t)D * 2 * D), bi = d2h_bf16(w->action_time_in_b, D);
+  std::vector<double> wa = d2h_bf16(w->action_in_w, (size_t)D * A), ba = d2h_bf16(w->action_in_b, D);
+  if (wi.empty() || bi.empty() || wa.empty() || ba.empty()) return RTVLA_ERR_CUDA;
+  std::vector<float> fold((size_t)D * A), tab((size_t)S * D);
+  std::vector<double> acc(A), e(D);
+  for (int n = 0; n < D; ++n) {
+    std::fill(acc.begin(), acc.end(), 0.0);
+    for (int i = 0; i < D; ++i) {
+      const double v = wi[(size_t)n * 2 * D + i];
+      for (int a = 0; a < A; ++a) acc[a] += v * wa[(size_t)i * A + a];
+    }
+    for (int a = 0; a < A; ++a) fold[(size_t)n * A + a] = (float)acc[a];
+  }
+  for (int k = 0; k < S; ++k) {
+    const double t = 1.0 - (double)k / S;
+    const int half = D / 2;
+    for (int i = 0; i < half; ++i) {
+      const double period = 4e-3 * std::pow(4.0 / 4e-3, (double)i / (half - 1));
+      const double ang = 2.0 * M_PI * t / period;
+      e[i] = std::sin(ang);
+      e[i + half] = std::cos(ang);
+    }
+    for (int n = 0; n < D; ++n) {
+      double v = bi[n];
+      for (int i = 0; i < D; ++i) v += wi[(size_t)n * 2 * D + i] * ba[i] + wi[(size_t)n * 2 * D + D + i] * e[i];
+      tab[(size_t)k * D + n] = (float)v;
+    }
+  }
+  if (cudaMemcpy(c->pi_wfold, fold.data(), fold.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(c->pi_ctab, tab.data(), tab.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+    return RTVLA_ERR_CUDA;
+  return RTVLA_OK;
+}
+
+// RoPE cos/sin tables: angle = pos * theta^(-2i/256) in fp64, rounded once to fp32
+rtvla_status build_rope(rtvla_ctx *c) {
   std::vector<float> rc((size_t)c->rope_rows * 128), rs((size_t)c->rope_rows * 128);
   for (int p = 0; p < c->rope_rows; ++p)
     for (int i = 0; i < 128; ++i) {
@@ -515,17 +628,24 @@ size_t max_attn_partials(int Bmax, int nq, int keys, int sm) {
 }
 
 bool weights_present(const rtvla_weights *w, const rtvla_config *cfg) {
-  if (!w->action_in_w || !w->action_in_b || !w->action_out_w || !w->action_out_b || !w->time_in_w ||
-      !w->time_in_b || !w->time_out_w || !w->time_out_b)
-    return false;
-  if (!w->wq || !w->wk || !w->wv || !w->wo || !w->wg || !w->wu || !w->wd || !w->ada_attn_w || !w->ada_attn_b ||
-      !w->ada_ffn_w || !w->ada_ffn_b)
-    return false;
+  const bool pi0 = cfg->variant == RTVLA_VARIANT_PI0;
+  if (!w->action_in_w || !w->action_in_b || !w->action_out_w || !w->action_out_b) return false;
+  if (!w->wq || !w->wk || !w->wv || !w->wo || !w->wg || !w->wu || !w->wd) return false;
   for (int l = 0; l < cfg->n_layers; ++l)
-    if (!w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->wg[l] || !w->wu[l] || !w->wd[l] ||
-        !w->ada_attn_w[l] || !w->ada_attn_b[l] || !w->ada_ffn_w[l] || !w->ada_ffn_b[l])
+    if (!w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->wg[l] || !w->wu[l] || !w->wd[l]) return false;
+  if (pi0) {
+    if (!w->state_w || !w->state_b || !w->action_time_in_w || !w->action_time_in_b || !w->action_time_out_w ||
+        !w->action_time_out_b || !w->ln1 || !w->ln2 || !w->final_ln)
       return false;
-  if (cfg->final_norm && (!w->ada_final_w || !w->ada_final_b)) return false;
+    for (int l = 0; l < cfg->n_layers; ++l)
+      if (!w->ln1[l] || !w->ln2[l]) return false;
+  } else {
+    if (!w->time_in_w || !w->time_in_b || !w->time_out_w || !w->time_out_b) return false;
+    if (!w->ada_attn_w || !w->ada_attn_b || !w->ada_ffn_w || !w->ada_ffn_b) return false;
+    for (int l = 0; l < cfg->n_layers; ++l)
+      if (!w->ada_attn_w[l] || !w->ada_attn_b[l] || !w->ada_ffn_w[l] || !w->ada_ffn_b[l]) return false;
+    if (cfg->final_norm && (!w->ada_final_w || !w->ada_final_b)) return false;
+  }
   if (cfg->has_prefill) {
     if (!w->pf_ln1 || !w->pf_wq || !w->pf_wk || !w->pf_wv || !w->pf_wo || !w->pf_ln2 || !w->pf_wg || !w->pf_wu ||
         !w->pf_wd)
@@ -573,6 +693,20 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
   }
   const double dt = -1.0 / S;  // Euler step folded into action_out_proj
   if (cudaMemcpy(c->w_in, w->action_in_w, (size_t)D * A * 2, dd) != cudaSuccess) return RTVLA_ERR_CUDA;
+  if (c->variant == RTVLA_VARIANT_PI0) {
+    c->pi_wfold = dalloc<float>(c, (size_t)D * A);
+    c->pi_ctab = dalloc<float>(c, (size_t)S * D);
+    c->pi_wato = dalloc<bf16>(c, (size_t)D * D);
+    c->pi_bato = dalloc<float>(c, D);
+    c->pi_wst = dalloc<bf16>(c, (size_t)D * A);
+    c->pi_bst = dalloc<float>(c, D);
+    if (!c->pi_wfold || !c->pi_ctab || !c->pi_wato || !c->pi_bato || !c->pi_wst || !c->pi_bst) return RTVLA_ERR_OOM;
+    if (cudaMemcpy(c->pi_wato, w->action_time_out_w, (size_t)D * D * 2, dd) != cudaSuccess ||
+        cudaMemcpy(c->pi_wst, w->state_w, (size_t)D * A * 2, dd) != cudaSuccess ||
+        launch_scale_to_f32(static_cast<const bf16 *>(w->action_time_out_b), D, 1.0, c->pi_bato, 0) != cudaSuccess ||
+        launch_scale_to_f32(static_cast<const bf16 *>(w->state_b), D, 1.0, c->pi_bst, 0) != cudaSuccess)
+      return RTVLA_ERR_CUDA;
+  }
   if (launch_scale_to_f32(static_cast<const bf16 *>(w->action_in_b), D, 1.0, c->b_in, 0) != cudaSuccess ||
       launch_scale_to_f32(static_cast<const bf16 *>(w->action_out_w), A * D, dt, c->w_out, 0) != cudaSuccess ||
       launch_scale_to_f32(static_cast<const bf16 *>(w->action_out_b), A, dt, c->b_out, 0) != cudaSuccess)
@@ -593,7 +727,9 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
   if (!c->s1p_attn || !c->gate_attn || !c->s1p_ffn || !c->gate_ffn || !c->bias_qkv || !c->bias_gu || !c->s1p_fin ||
       !c->shift_fin || !c->rope_cos || !c->rope_sin)
     return RTVLA_ERR_OOM;
-  rtvla_status st = build_tables(c, w);
+  rtvla_status st = c->variant == RTVLA_VARIANT_PI0 ? build_tables_pi0(c, w) : build_tables(c, w);
+  if (st != RTVLA_OK) return st;
+  st = build_rope(c);
   if (st != RTVLA_OK) return st;
 
   // ---- prefix-pass weights, Gemma RMSNorm (1 + w) folded into the following projection
@@ -663,7 +799,8 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
     return RTVLA_ERR_CUDA;
 
   // ---- tensor maps (weights: 128-row boxes; activations: one map per token-tile height)
-  bool ok = make_map(&c->tm_wqkv, c->w_qkv, (uint64_t)L * 2560, D, 128) &&
+  bool ok = (c->variant != RTVLA_VARIANT_PI0 || make_map(&c->tm_wato, c->pi_wato, D, D, 128)) &&
+            make_map(&c->tm_wqkv, c->w_qkv, (uint64_t)L * 2560, D, 128) &&
             make_map(&c->tm_wo, c->w_o, (uint64_t)L * D, NQH * HD, 128) &&
             make_map(&c->tm_wgu, c->w_gu, (uint64_t)L * 2 * F, D, 128) &&
             make_map(&c->tm_wd, c->w_d, (uint64_t)L * D, F, 128) && make_xmaps(&c->tm_op, c->op, M, D) &&
@@ -683,7 +820,7 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
 
   // ---- persistent engine (batch 1, chunk <= 64): norm statistics and attention partials
   if (persistent_init_attributes() != cudaSuccess) return RTVLA_ERR_CUDA;
-  c->pers_ok = C <= 64 && persistent_fits(c->sm_count);
+  c->pers_ok = c->variant == RTVLA_VARIANT_PI05 && C <= 64 && persistent_fits(c->sm_count);
   if (c->pers_ok) {
     const int sp = persistent_max_splits(c->sm_count);
     c->ss_attn = dalloc<float>(c, 64);
@@ -747,6 +884,7 @@ const char *rtvla_status_string(rtvla_status s) {
     case RTVLA_ERR_DEVICE_TIMEOUT: return "a bounded device wait expired";
     case RTVLA_ERR_UNSUPPORTED: return "unsupported model shape or engine";
     case RTVLA_ERR_DEVICE_BOUNDS: return "a valid length exceeded its buffer";
+    case RTVLA_ERR_GUARD_OVERWRITE: return "a guard band around a library buffer was overwritten";
   }
   return "unknown status";
 }
@@ -766,11 +904,23 @@ rtvla_status rtvla_create(const rtvla_weights *w, const rtvla_config *cfg, rtvla
   c->cfg = *cfg;
   c->L = cfg->n_layers;
   c->S = cfg->n_steps;
-  c->C = cfg->chunk;
+  c->variant = cfg->variant;
+  c->first = cfg->variant == RTVLA_VARIANT_PI0 ? 1 : 0;
+  if (c->variant == RTVLA_VARIANT_PI0) c->cfg.final_norm = 1;  // π0 ends in an RMSNorm
+  c->Ca = cfg->chunk;
+  c->C = cfg->chunk + c->first;
   c->Bmax = cfg->max_batch;
   c->Pmax = cfg->max_prefix;
   c->engine = cfg->engine;
+  if (const char *env = std::getenv("RTVLA_CHECKED")) c->checked = std::atoi(env) != 0;
+  if (const char *env = std::getenv("RTVLA_DEVICE_MEMORY_CAP")) c->mem_cap = (size_t)std::strtoull(env, nullptr, 10);
   rtvla_status st = create_impl(c, w);
+  if (st == RTVLA_OK && c->checked) {
+    const size_t b = c->guards.size() * sizeof(GuardRegion);
+    if (cudaMalloc(&c->d_guards, b) != cudaSuccess ||
+        cudaMemcpy(c->d_guards, c->guards.data(), b, cudaMemcpyHostToDevice) != cudaSuccess)
+      st = RTVLA_ERR_CUDA;
+  }
   if (st != RTVLA_OK) {
     cudaGetLastError();
     free_all(c);
@@ -818,15 +968,15 @@ static CallArgs host_args(const rtvla_kv *kv) {
   return a;
 }
 
-rtvla_status rtvla_sample_actions(rtvla_ctx *c, const float *noise, const rtvla_kv *kv, float *actions_out,
-                                  void *stream) {
-  if (!c || !noise || !actions_out) return RTVLA_ERR_INVALID_ARG;
+static rtvla_status sample_impl(rtvla_ctx *c, const float *noise, const float *state, const rtvla_kv *kv,
+                                float *actions_out, void *stream) {
   rtvla_status s = check_kv(c, kv);
   if (s != RTVLA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CallArgs a = host_args(kv);
   a.noise = noise;
   a.actions = actions_out;
+  a.state = state;
   if (c->engine == RTVLA_ENGINE_PERSISTENT && !use_persistent(c, kv->batch)) return RTVLA_ERR_UNSUPPORTED;
   if (use_persistent(c, kv->batch)) {
     if (cudaMemcpyAsync(c->args_dn, &a, sizeof(a), cudaMemcpyHostToDevice, st) != cudaSuccess) return RTVLA_ERR_CUDA;
@@ -851,6 +1001,20 @@ rtvla_status rtvla_sample_actions(rtvla_ctx *c, const float *noise, const rtvla_
   return RTVLA_OK;
 }
 
+rtvla_status rtvla_sample_actions(rtvla_ctx *c, const float *noise, const rtvla_kv *kv, float *actions_out,
+                                  void *stream) {
+  if (!c || !noise || !actions_out) return RTVLA_ERR_INVALID_ARG;
+  if (c->variant != RTVLA_VARIANT_PI05) return RTVLA_ERR_INVALID_ARG;  // π0 needs the state
+  return sample_impl(c, noise, nullptr, kv, actions_out, stream);
+}
+
+rtvla_status rtvla_sample_actions_pi0(rtvla_ctx *c, const float *noise, const float *state, const rtvla_kv *kv,
+                                      float *actions_out, void *stream) {
+  if (!c || !noise || !state || !actions_out) return RTVLA_ERR_INVALID_ARG;
+  if (c->variant != RTVLA_VARIANT_PI0) return RTVLA_ERR_UNSUPPORTED;
+  return sample_impl(c, noise, state, kv, actions_out, stream);
+}
+
 rtvla_status rtvla_sample_actions_host(rtvla_ctx *c, const float *noise, const void *kv_k, const void *kv_v,
                                        const int32_t *valid_len, int batch, int prefix_cap, float *actions_out,
                                        void *stream) {
@@ -859,7 +1023,7 @@ rtvla_status rtvla_sample_actions_host(rtvla_ctx *c, const float *noise, const v
   if (batch > c->Bmax || prefix_cap > c->Pmax) return RTVLA_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t kv_elems = (size_t)c->L * batch * prefix_cap * HD;
-  const size_t io = (size_t)batch * c->C * A;
+  const size_t io = (size_t)batch * c->Ca * A;
   if (kv_elems > c->st_kv_elems) {
     if (c->st_k) cudaFree(c->st_k);
     if (c->st_v) cudaFree(c->st_v);
@@ -943,6 +1107,12 @@ rtvla_status rtvla_prefill(rtvla_ctx *c, const void *prefix_embeds, const uint8_
 
 rtvla_status rtvla_sync_status(rtvla_ctx *c, void *stream) {
   if (!c) return RTVLA_ERR_INVALID_ARG;
+  if (c->checked &&
+      launch_check_guards(c->d_guards, (int)c->guards.size(), c->ctl, static_cast<cudaStream_t>(stream)) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return RTVLA_ERR_CUDA;
+  }
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return RTVLA_ERR_CUDA;
@@ -954,12 +1124,28 @@ rtvla_status rtvla_sync_status(rtvla_ctx *c, void *stream) {
   if (cudaMemcpy(c->ctl, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return RTVLA_ERR_CUDA;
   if (h.err & DEVERR_TIMEOUT) return RTVLA_ERR_DEVICE_TIMEOUT;
   if (h.err & DEVERR_MASK) return RTVLA_ERR_MASK_NOT_PREFIX;
+  if (h.err & DEVERR_GUARD) return RTVLA_ERR_GUARD_OVERWRITE;
   return RTVLA_ERR_DEVICE_BOUNDS;
 }
 
-rtvla_status rtvla_debug_trace(rtvla_ctx *c, const float *noise, const rtvla_kv *kv, int step, float *h_layers,
-                               void *stream) {
-  if (!c || !noise || !h_layers) return RTVLA_ERR_INVALID_ARG;
+rtvla_status rtvla_debug_plant_guard_fault(rtvla_ctx *c) {
+  if (!c) return RTVLA_ERR_INVALID_ARG;
+  if (!c->checked) return RTVLA_ERR_UNSUPPORTED;
+  for (const GuardRegion &g : c->guards)
+    if (g.base + GUARD_BYTES == reinterpret_cast<unsigned char *>(c->h)) {
+      // the first byte past the end of the residual-stream buffer, as a kernel writing one
+      // row too far would touch it
+      if (cudaDeviceSynchronize() != cudaSuccess || cudaMemset(g.base + GUARD_BYTES + g.bytes, 0, 1) != cudaSuccess) {
+        cudaGetLastError();
+        return RTVLA_ERR_CUDA;
+      }
+      return RTVLA_OK;
+    }
+  return RTVLA_ERR_UNSUPPORTED;
+}
+
+static rtvla_status trace_impl(rtvla_ctx *c, const float *noise, const float *state, const rtvla_kv *kv, int step,
+                               float *h_layers, void *stream) {
   rtvla_status s = check_kv(c, kv);
   if (s != RTVLA_OK) return s;
   if (step < 0 || step >= c->S) return RTVLA_ERR_INVALID_ARG;
@@ -967,11 +1153,35 @@ rtvla_status rtvla_debug_trace(rtvla_ctx *c, const float *noise, const rtvla_kv 
   CallArgs a = host_args(kv);
   a.noise = noise;
   a.actions = nullptr;
+  a.state = state;
+  if (c->engine == RTVLA_ENGINE_PERSISTENT && !use_persistent(c, kv->batch)) return RTVLA_ERR_UNSUPPORTED;
   if (cudaMemcpyAsync(c->args_tr, &a, sizeof(a), cudaMemcpyHostToDevice, st) != cudaSuccess) return RTVLA_ERR_CUDA;
+  if (use_persistent(c, kv->batch)) {
+    // the engine rtvla_sample_actions would run: the persistent kernel, recording h at `step`
+    if (launch_persistent(c, c->args_tr, kv, st, h_layers, step) != cudaSuccess) {
+      cudaGetLastError();
+      return RTVLA_ERR_CUDA;
+    }
+    return RTVLA_OK;
+  }
   int n = 0;
   if (enqueue_denoise(c, c->args_tr, kv->batch, kv->prefix_cap, st, h_layers, step, &n) != cudaSuccess)
     return RTVLA_ERR_CUDA;
   return RTVLA_OK;
+}
+
+rtvla_status rtvla_debug_trace(rtvla_ctx *c, const float *noise, const rtvla_kv *kv, int step, float *h_layers,
+                               void *stream) {
+  if (!c || !noise || !h_layers) return RTVLA_ERR_INVALID_ARG;
+  if (c->variant != RTVLA_VARIANT_PI05) return RTVLA_ERR_INVALID_ARG;
+  return trace_impl(c, noise, nullptr, kv, step, h_layers, stream);
+}
+
+rtvla_status rtvla_debug_trace_pi0(rtvla_ctx *c, const float *noise, const float *state, const rtvla_kv *kv, int step,
+                                   float *h_layers, void *stream) {
+  if (!c || !noise || !state || !h_layers) return RTVLA_ERR_INVALID_ARG;
+  if (c->variant != RTVLA_VARIANT_PI0) return RTVLA_ERR_UNSUPPORTED;
+  return trace_impl(c, noise, state, kv, step, h_layers, stream);
 }
 
 int rtvla_kernels_per_call(rtvla_ctx *c, int batch) {
@@ -1041,9 +1251,9 @@ extern "C" rtvla_status rtvla_sample_actions_host_static(rtvla_ctx *c, const flo
   if (!c || !noise || !kv_k || !kv_v || !valid_len || !actions_out) return RTVLA_ERR_INVALID_ARG;
   if (batch < 1 || prefix_cap < 1) return RTVLA_ERR_INVALID_ARG;
   if (batch > c->Bmax || prefix_cap > c->Pmax) return RTVLA_ERR_SHAPE;
-  if (c->engine == RTVLA_ENGINE_PERSISTENT) return RTVLA_ERR_UNSUPPORTED;
+  if (c->engine == RTVLA_ENGINE_PERSISTENT && !use_persistent(c, batch)) return RTVLA_ERR_UNSUPPORTED;
   const size_t kv_elems = (size_t)c->L * batch * prefix_cap * HD;
-  const size_t io = (size_t)batch * c->C * A;
+  const size_t io = (size_t)batch * c->Ca * A;
   const size_t off_act = round256(io * 4);
   const size_t off_vl = off_act + round256(io * 4);
   const size_t off_k = off_vl + round256((size_t)batch * 4);
@@ -1079,10 +1289,23 @@ extern "C" rtvla_status rtvla_sample_actions_host_static(rtvla_ctx *c, const flo
   a.batch = batch;
   a.cap = prefix_cap;
   if (cudaMemcpyAsync(c->args_dn, &a, sizeof(a), hd, st) != cudaSuccess) return RTVLA_ERR_CUDA;
-  // A graph already captured for this shape is replayed; otherwise the same kernels are
-  // launched directly, so that this call never instantiates anything.
+  // The engine rtvla_sample_actions would pick: the persistent kernel (one launch, nothing
+  // allocated: its per-call tensor maps are encoded on the host); else a graph already
+  // captured for this shape is replayed; otherwise the same kernels are launched directly,
+  // so that this call never instantiates anything.
   auto it = c->graphs_dn.find(std::make_pair(batch, prefix_cap));
-  if (it != c->graphs_dn.end()) {
+  if (use_persistent(c, batch)) {
+    rtvla_kv kv;
+    kv.k = d_k;
+    kv.v = d_v;
+    kv.valid_len = d_vl;
+    kv.batch = batch;
+    kv.prefix_cap = prefix_cap;
+    if (launch_persistent(c, c->args_dn, &kv, st) != cudaSuccess) {
+      cudaGetLastError();
+      return RTVLA_ERR_CUDA;
+    }
+  } else if (it != c->graphs_dn.end()) {
     if (cudaGraphLaunch(it->second.exec, st) != cudaSuccess) return RTVLA_ERR_CUDA;
   } else {
     int n = 0;

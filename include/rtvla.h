@@ -46,7 +46,8 @@ typedef enum {
   RTVLA_ERR_CUDA = 5,            /* a CUDA runtime call failed; the context may be unusable */
   RTVLA_ERR_DEVICE_TIMEOUT = 6,  /* a bounded device-side wait expired (device-detected) */
   RTVLA_ERR_UNSUPPORTED = 7,     /* model shape the kernels are not built for */
-  RTVLA_ERR_DEVICE_BOUNDS = 8    /* a valid length exceeded its buffer (device-detected, clamped) */
+  RTVLA_ERR_DEVICE_BOUNDS = 8,   /* a valid length exceeded its buffer (device-detected, clamped) */
+  RTVLA_ERR_GUARD_OVERWRITE = 9  /* checked mode: a guard band around a library buffer changed */
 } rtvla_status;
 
 /* Engines that run the denoise loop (rtvla_config.engine).  The persistent engine applies to
@@ -59,6 +60,17 @@ enum {
   RTVLA_ENGINE_LAYERED = 1,    /* one kernel per phase, the whole loop captured as one CUDA graph */
   RTVLA_ENGINE_PERSISTENT = 2  /* one persistent kernel per call; calls it cannot serve return
                                   RTVLA_ERR_UNSUPPORTED */
+};
+
+/* Model variants (rtvla_config.variant).  [PAPER] Sec. 1.1.2 and the "Running VLAs at
+ * Real-time Speed" summary ("How": the action time encoder): π0 routes the robot state and
+ * the noisy actions to the action expert; π0.5 conditions the expert on the time through
+ * AdaRMS [BLOG "pi0.5 inference flow"]. */
+enum {
+  RTVLA_VARIANT_PI05 = 0, /* AdaRMS (scale, shift, gate) from the time MLP; gated residuals */
+  RTVLA_VARIANT_PI0 = 1   /* suffix = [state token ; actions]; action tokens from the action-time
+                             MLP; plain RMSNorm (scale 1 + w); ungated residuals; final norm.
+                             Runs on the layered engine (AUTO picks it; PERSISTENT is refused) */
 };
 
 /*
@@ -86,6 +98,7 @@ typedef struct {
   int engine;      /* RTVLA_ENGINE_* */
   float rms_eps;   /* 1e-6 */
   float rope_theta;/* 10000 */
+  int variant;     /* RTVLA_VARIANT_* (0 = π0.5) */
 } rtvla_config;
 
 /*
@@ -126,6 +139,17 @@ typedef struct {
   const void *const *pf_wg;  /* [L] -> [Fp][Dp] */
   const void *const *pf_wu;  /* [L] -> [Fp][Dp] */
   const void *const *pf_wd;  /* [L] -> [Dp][Fp] */
+  /* π0 (variant RTVLA_VARIANT_PI0; then time_in_*, ada_* are not read, action_in_* and
+   * action_out_* are) */
+  const void *state_w;           /* [D][A]   state_proj */
+  const void *state_b;           /* [D] */
+  const void *action_time_in_w;  /* [D][2D]  action_time_mlp_in over [action_in_proj(x) ; SinEmb(t)] */
+  const void *action_time_in_b;  /* [D] */
+  const void *action_time_out_w; /* [D][D]   action_time_mlp_out */
+  const void *action_time_out_b; /* [D] */
+  const void *const *ln1;        /* [L] -> [D]  input_layernorm weight w (scale 1 + w) */
+  const void *const *ln2;        /* [L] -> [D]  post_attention_layernorm weight w */
+  const void *final_ln;          /* [D]        final norm weight w */
 } rtvla_weights;
 
 /*
@@ -180,6 +204,22 @@ rtvla_status rtvla_sample_actions(rtvla_ctx *ctx, const float *noise, const rtvl
                                   float *actions_out, void *stream);
 
 /*
+ * The π0 denoise loop (context variant RTVLA_VARIANT_PI0) [PAPER summary, "How"; Sec. 1.1.2]:
+ * each step builds the suffix [state token ; C action tokens] — state token = state_proj(state);
+ * action token = action_time_mlp_out(SiLU(action_time_mlp_in([action_in_proj(x) ; SinEmb(t)]))),
+ * computed as SiLU(W_fold x + c_k) with W_fold = action_time_mlp_in[:, :D] @ action_in_proj and
+ * the 10 rows c_k tabulated at create time — runs the L layers over those C + 1 tokens
+ * (plain RMSNorm, ungated residuals; every suffix token sees every valid prefix key and every
+ * suffix token, at positions Lv + i with the state at i = 0), then a final RMSNorm and
+ * action_out_proj on the action tokens, and x += dt * v.  noise, actions_out: device f32
+ * [batch][chunk][action_dim]; state: device f32 [batch][action_dim].  Errors: INVALID_ARG,
+ * SHAPE, UNSUPPORTED (a π0.5 context, or engine PERSISTENT); device-detected errors through
+ * rtvla_sync_status.  rtvla_sample_actions on a π0 context returns INVALID_ARG (no state).
+ */
+rtvla_status rtvla_sample_actions_pi0(rtvla_ctx *ctx, const float *noise, const float *state,
+                                      const rtvla_kv *kv, float *actions_out, void *stream);
+
+/*
  * Same loop from host buffers: copies noise (host f32 [batch][chunk][action_dim]), the
  * cache (host bf16 k and v [n_layers][batch][prefix_cap][head_dim], host int32 valid_len
  * [batch]) to the context's device staging, runs the loop, copies the actions back to
@@ -201,18 +241,24 @@ rtvla_status rtvla_sample_actions_host(rtvla_ctx *ctx, const float *noise, const
  * rtvla_sample_actions_host allocates its device staging on first use.  This call allocates
  * nothing: it stages the inputs and outputs in one file-scope device array of 32 MiB
  * (RTVLA_STATIC_STAGING_BYTES) that every GPU loading this library holds until the process
- * exits, and it captures no graph (a graph already captured for this shape by
- * rtvla_sample_actions is replayed; otherwise the kernels are launched directly).
+ * exits, and it captures no graph.  It runs the engine rtvla_sample_actions would run: the
+ * persistent kernel where it applies (batch 1, chunk <= 64, engine AUTO or PERSISTENT);
+ * otherwise a layered graph already captured for this shape by rtvla_sample_actions is
+ * replayed, and without one the layered kernels are launched directly (slower: one launch
+ * per kernel).
  *
  * Arguments, layout and result are those of rtvla_sample_actions_host (host buffers, the
  * call waits for `stream`).  The device of `ctx` must be current.  Errors: INVALID_ARG;
  * SHAPE when batch or prefix_cap exceed the context's capacity or when noise + actions +
  * valid_len + K + V (each rounded up to 256 bytes) need more than 32 MiB, checked before
- * anything is copied; UNSUPPORTED for the persistent engine; CUDA.
+ * anything is copied; UNSUPPORTED when the engine is PERSISTENT and the call is one it
+ * cannot serve; CUDA.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress);
  * make that first call before any stream capture.  All calls share the one array, which
  * keeps the last call's contents (every byte a call reads is written by that call first):
  * calls that overlap on the GPU — from two streams or two contexts on one device — race.
+ * The call also writes the context's device argument block, which rtvla_sample_actions and
+ * its graphs read: it must not overlap any other sample call on the same context either.
  */
 rtvla_status rtvla_sample_actions_host_static(rtvla_ctx *ctx, const float *noise, const void *kv_k,
                                               const void *kv_v, const int32_t *valid_len, int batch,
@@ -220,17 +266,42 @@ rtvla_status rtvla_sample_actions_host_static(rtvla_ctx *ctx, const float *noise
 
 /*
  * Waits for `stream`, then reads and clears the device error word: RTVLA_OK, or the first
- * device-detected error (DEVICE_TIMEOUT, DEVICE_BOUNDS, MASK_NOT_PREFIX) since the last call.
+ * device-detected error (DEVICE_TIMEOUT, DEVICE_BOUNDS, MASK_NOT_PREFIX, GUARD_OVERWRITE)
+ * since the last call.
+ *
+ * Checked mode (a run-time race and bounds detector; no counterpart on the pages): with the
+ * environment variable RTVLA_CHECKED=1 when rtvla_create runs, every buffer the context
+ * allocates sits between two 4096-byte guard bands filled with 0xA5, and this call first
+ * enqueues a check of every band on `stream`; a band that changed (a kernel wrote past a
+ * buffer) is refilled and reported as RTVLA_ERR_GUARD_OVERWRITE.  A device-memory cap for
+ * the context can be set with RTVLA_DEVICE_MEMORY_CAP=<bytes>: rtvla_create then returns
+ * RTVLA_ERR_OOM, having freed everything, when the context would need more.
  */
 rtvla_status rtvla_sync_status(rtvla_ctx *ctx, void *stream);
 
 /*
- * Test hook: runs the loop up to and including step `step` (0-based) with the layered
- * engine and writes the expert hidden state of that step before layer 0 and after each
- * layer to h_layers: device f32 [n_layers + 1][batch][chunk][width].  Asynchronous.
+ * Test hook of checked mode: overwrites the first byte after the context's residual-stream
+ * buffer (the kind of write a kernel that runs one row too far makes), so that the next
+ * rtvla_sync_status must report RTVLA_ERR_GUARD_OVERWRITE.  Synchronous.  Errors:
+ * INVALID_ARG; UNSUPPORTED when the context is not in checked mode; CUDA.
+ */
+rtvla_status rtvla_debug_plant_guard_fault(rtvla_ctx *ctx);
+
+/*
+ * Test hook: runs the loop with the engine rtvla_sample_actions would run for this call and
+ * writes the expert hidden state of step `step` (0-based) before layer 0 and after each
+ * layer to h_layers: device f32 [n_layers + 1][batch][chunk][width].  The persistent engine
+ * runs the whole loop and records the step on the way; the layered engine stops after it.
+ * No actions are written.  Asynchronous.  Errors: INVALID_ARG, SHAPE, UNSUPPORTED (engine
+ * PERSISTENT and a call it cannot serve), CUDA.
  */
 rtvla_status rtvla_debug_trace(rtvla_ctx *ctx, const float *noise, const rtvla_kv *kv, int step,
                                float *h_layers, void *stream);
+
+/* The test hook of rtvla_debug_trace for a π0 context (state: device f32 [batch][action_dim]);
+ * h_layers is device f32 [n_layers + 1][batch][chunk + 1][width], the state token first. */
+rtvla_status rtvla_debug_trace_pi0(rtvla_ctx *ctx, const float *noise, const float *state,
+                                   const rtvla_kv *kv, int step, float *h_layers, void *stream);
 
 /* Number of kernels of this library one rtvla_sample_actions call launches at `batch`
  * with the context's engine (after the call has been made once at that batch). */

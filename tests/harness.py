@@ -15,6 +15,14 @@ ACT_MAX_ABS = 3e-2
 ACT_REL_L2 = 1e-2
 H_REL_L2 = 1e-2
 KV_REL_L2 = 1e-2
+# Per-layer hidden states and updates of networks whose residual updates are O(1) (the
+# "stressed" weights with AdaRMS gate 1, and the ungated pi0 expert) at full size: relative L2
+# 2e-2.  There every layer adds an O(1) update computed from bf16 operands (bf16 Q and K at
+# attention logits of magnitude ~10 alone move an update by ~1e-2), and 18 such layers carry
+# it: measured on B200, 1.00e-2 to 1.07e-2 at the worst layer, on both engines.  Every planted
+# mistake moves them by 0.33 or more (tests/test_oracle_pins.py).  The plain-weight workloads
+# keep the 1e-2 bound.
+O1_REL_L2 = 2e-2
 
 
 def rel_l2(a, b) -> float:
@@ -36,7 +44,7 @@ class GpuModel:
 
     def __init__(self, wl: WL.Workload, expert_bits: dict, prefill_bits: dict | None = None,
                  max_batch: int | None = None, max_prefix: int | None = None, engine: int = R.ENGINE_AUTO,
-                 final_norm: bool | None = None):
+                 final_norm: bool | None = None, variant: int = R.VARIANT_PI05):
         dev = {k: bf16_dev(v) for k, v in expert_bits.items()}
         if prefill_bits is not None:
             dev.update({k: bf16_dev(v) for k, v in prefill_bits.items()})
@@ -44,7 +52,7 @@ class GpuModel:
         self.cfg = R.make_config(n_layers=s.n_layers, chunk=wl.chunk, max_prefix=max_prefix or wl.prefix_cap,
                                  max_batch=max_batch or wl.batch, n_steps=s.n_steps,
                                  final_norm=s.final_norm if final_norm is None else final_norm,
-                                 has_prefill=prefill_bits is not None, engine=engine)
+                                 has_prefill=prefill_bits is not None, engine=engine, variant=variant)
         self.ctx = R.rtvla_create(dev, self.cfg)
         del dev
         torch.cuda.synchronize()
@@ -85,6 +93,26 @@ class GpuModel:
         assert st == 0, R.STATUS[st]
         return h.cpu().numpy()
 
+    def sample_pi0(self, noise: np.ndarray, state: np.ndarray, k, v, valid) -> np.ndarray:
+        B, C, A = noise.shape
+        x = torch.from_numpy(np.ascontiguousarray(noise, dtype=np.float32)).cuda()
+        s = torch.from_numpy(np.ascontiguousarray(state, dtype=np.float32)).cuda()
+        out = torch.empty_like(x)
+        R.rtvla_sample_actions_pi0(self.ctx, x, s, self.kv(k, v, valid, B, k.shape[2]), out)
+        st = R.rtvla_sync_status(self.ctx)
+        assert st == 0, R.STATUS[st]
+        return out.cpu().numpy()
+
+    def trace_pi0(self, noise: np.ndarray, state: np.ndarray, k, v, valid, step: int) -> np.ndarray:
+        B, C, A = noise.shape
+        x = torch.from_numpy(np.ascontiguousarray(noise, dtype=np.float32)).cuda()
+        s = torch.from_numpy(np.ascontiguousarray(state, dtype=np.float32)).cuda()
+        h = torch.empty((self.cfg.n_layers + 1, B, C + 1, 1024), dtype=torch.float32, device="cuda")
+        R.rtvla_debug_trace_pi0(self.ctx, x, s, self.kv(k, v, valid, B, k.shape[2]), step, h)
+        st = R.rtvla_sync_status(self.ctx)
+        assert st == 0, R.STATUS[st]
+        return h.cpu().numpy()
+
     def prefill(self, emb_bits: np.ndarray, mask: np.ndarray, cap: int | None = None):
         B, P, _ = emb_bits.shape
         cap = cap or P
@@ -112,14 +140,17 @@ def assert_actions_close(gpu, ref, what=""):
     return d, r
 
 
-def assert_trace_close(gpu_tr, ref_tr, what=""):
-    worst = 0.0
+def assert_trace_close(gpu_tr, ref_tr, what="", tol=H_REL_L2):
+    """Every hidden state and every layer's update within relative L2 tol; returns (worst
+    hidden-state error, worst update error)."""
+    worst_h = worst_u = 0.0
+    upd_tol = tol
     for i in range(ref_tr.shape[0]):
         r = rel_l2(gpu_tr[i], ref_tr[i])
-        worst = max(worst, r)
-        assert r <= H_REL_L2, f"{what}: hidden state {i} rel-L2 {r:.3e}"
+        worst_h = max(worst_h, r)
+        assert r <= tol, f"{what}: hidden state {i} rel-L2 {r:.3e}"
         if i > 0:
             dr = rel_l2(gpu_tr[i] - gpu_tr[i - 1], ref_tr[i] - ref_tr[i - 1])
-            worst = max(worst, dr)
-            assert dr <= H_REL_L2, f"{what}: layer {i - 1} update rel-L2 {dr:.3e}"
-    return worst
+            worst_u = max(worst_u, dr)
+            assert dr <= upd_tol, f"{what}: layer {i - 1} update rel-L2 {dr:.3e}"
+    return worst_h, worst_u

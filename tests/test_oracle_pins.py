@@ -495,39 +495,44 @@ def test_golden_regression_of_the_oracle():
 
 
 # The same planted mistakes at full size (18 layers, width 1024, 1-view: chunk 50, 280 of 288
-# prefix tokens valid) with PLAIN N(0, 0.02) weights, caught by the per-layer check the GPU
-# tests apply (every layer's hidden state and update within relative L2 1e-2).  On plain
-# weights a check of the final actions alone misses several of them, because each layer's
-# update is small next to h; the per-layer updates are not.  Step 0 of the loop is traced
-# (the trace of step 0 depends only on t_0 = 1, so one Euler step suffices).
+# prefix tokens valid), on plain N(0, 0.02) and on stressed weights, caught by the per-layer
+# check the GPU tests apply (every hidden state and every layer's update within the bound of
+# PER_LAYER_TOL).  On plain weights a check of the final actions alone misses
+# several of them, because each layer's update is small next to h; the per-layer updates do
+# not.  Step 0 of the loop is traced (it depends only on t_0 = 1: one Euler step suffices).
 
-@pytest.fixture(scope="module")
-def plain_full_size():
+@pytest.fixture(scope="module", params=["plain", "stressed"])
+def full_size(request):
     from dataclasses import replace
     w = WL.workload(2)
     one = replace(w.expert, n_steps=1)
-    Wt = M.Weights(WL.as_f32(WL.expert_weights(w.expert)))
+    Wt = M.Weights(WL.as_f32(WL.expert_weights(w.expert, stressed=request.param == "stressed")))
     k, v, lv = WL.kv_cache(w)
     kf, vf = gen.bf16_to_f32(k), gen.bf16_to_f32(v)
     x0 = WL.noise(w)
     _, tr = M.sample_actions(Wt, one, x0, kf, vf, lv, trace_step=0)
-    return one, Wt, kf, vf, lv, x0, tr
+    return request.param, one, Wt, kf, vf, lv, x0, tr
 
 
-def _fails_per_layer(tr, rtr):
-    return any(rel_l2(tr[i], rtr[i]) > H_REL_L2 for i in range(tr.shape[0])) or any(
-        rel_l2(tr[i] - tr[i - 1], rtr[i] - rtr[i - 1]) > H_REL_L2 for i in range(1, tr.shape[0]))
+# the per-layer bound of the GPU tests (hidden states and updates): 1e-2 on plain weights;
+# 2e-2 where updates are O(1) (stressed weights), there the bf16 floor of the GPU path is ~1e-2
+PER_LAYER_TOL = {"plain": 1e-2, "stressed": 2e-2}
+
+
+def _fails_per_layer(tr, rtr, tol):
+    return any(rel_l2(tr[i], rtr[i]) > tol for i in range(tr.shape[0])) or any(
+        rel_l2(tr[i] - tr[i - 1], rtr[i] - rtr[i - 1]) > tol for i in range(1, tr.shape[0]))
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS) + ["valid_len_plus_one"])
-def test_mutants_fail_the_per_layer_check_at_full_size(plain_full_size, monkeypatch, name):
-    one, Wt, kf, vf, lv, x0, rtr = plain_full_size
+def test_mutants_fail_the_per_layer_check_at_full_size(full_size, monkeypatch, name):
+    kind, one, Wt, kf, vf, lv, x0, rtr = full_size
     if name == "valid_len_plus_one":
         _, tr = M.sample_actions(Wt, one, x0, kf, vf, lv + 1, trace_step=0)
     else:
         MUTANTS[name](monkeypatch)
         _, tr = M.sample_actions(Wt, one, x0, kf, vf, lv, trace_step=0)
-    assert _fails_per_layer(tr, rtr), name
+    assert _fails_per_layer(tr, rtr, PER_LAYER_TOL[kind]), (kind, name)
 
 
 # ---------------------------------------------------------------------------------------
