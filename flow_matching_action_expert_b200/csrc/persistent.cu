@@ -30,19 +30,19 @@ namespace pk {
 constexpr int THREADS = 320;
 constexpr int NCOMP = 256;
 constexpr int RING = 5;
-constexpr int PREFETCH = 24;              // weight tiles the L2 prefetch cursor runs ahead of the ring
 constexpr int WST = 128 * 128;            // one 128-row x 64-column bf16 weight tile
-constexpr int NOPK = 8;                   // operand K blocks per unit, at most (64 tokens x 64 bf16, 128B swizzle)
-constexpr int STG = 8192;                 // one staged fp32 tile: 64 rows x 32 columns, 128B swizzle
-constexpr int STAGE = 16 * STG;           // a unit's whole fp32 K slice (128 KB), converted in place
-constexpr int NSTB = 8;                   // staging barriers (one per K block or per pair of K blocks)
+constexpr int NOPK = 8;                   // operand K blocks (64 tokens x 64 bf16 each, 128B swizzle)
+constexpr int OPB = NOPK * 8192;
+constexpr int NGRP = 2;                   // fp32 staging groups (double buffer)
+constexpr int STG = 8192;                 // one staged tile: 64 rows x 32 columns, 128B swizzle
+constexpr int GRPB = 4 * STG;             // a group: 4 tiles, filled by one or two 3-D TMA boxes
 constexpr int TBL = 4096;                 // per-unit slice of the AdaRMS scale / GELU bias tables
-constexpr int REGION = STAGE + TBL;       // staging / operands + table | attention | epilogue tile
+constexpr int REGION = OPB + NGRP * GRPB + TBL;  // operands + staging + table | attention | epilogue tile
 constexpr int LDS = 264;                  // attention shared rows (bf16), 528 bytes
 constexpr int KC = 32;                    // attention keys per chunk
 constexpr int ATT_BYTES = (64 + 2 * KC) * LDS * 2;
 static_assert(ATT_BYTES <= REGION, "attention tiles must fit the shared region");
-constexpr int NBARS = 2 * RING + NOPK + NSTB + 4;
+constexpr int NBARS = 2 * RING + NOPK + NGRP + 4;
 constexpr int SMEM = RING * WST + REGION + 1024 + NBARS * 8 + 64;
 constexpr int D = 1024, F = 4096, HD = 256, NH = 8, A = 32;
 constexpr int MAXSPLIT = 18;
@@ -54,9 +54,6 @@ __device__ __forceinline__ int kb_total(int kind) { return kind == QKV || kind =
 __device__ __forceinline__ int k_splits(int kind) { return kind == QKV ? 7 : (kind == GU ? 2 : 18); }
 __device__ __forceinline__ int units(int kind) { return n_tiles(kind) * k_splits(kind); }
 __device__ __forceinline__ int rows_per_layer(int kind) { return kind == QKV ? 2560 : (kind == GU ? 8192 : 1024); }
-// bytes between the operand K blocks of a unit: each K block is converted in place inside the
-// fp32 staging of its columns (h: 64 x 64 fp32; gate and up accumulators: twice that)
-__device__ __forceinline__ int slot_bytes(int kind) { return kind == DN ? 4 * STG : 2 * STG; }
 __device__ __forceinline__ int rotation(int gp, int ncta) { return (gp * 37) % ncta; }
 __device__ __forceinline__ int first_unit(int gp, int c, int ncta) {
   return (c - rotation(gp, ncta) + ncta) % ncta;
@@ -130,8 +127,6 @@ __device__ __forceinline__ void grid_sync(const PersistParams &p, unsigned *bar,
     fence_proxy_async_global();
     stamp(p, epoch, 7);
     ++epoch;
-    // release-ordered arrival without a return value: the poll below starts at once instead
-    // of after the atomic's round trip
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar + 32 * (blockIdx.x % NBC)) : "memory");
     if (!bar_passed(bar, epoch, ncta)) {
       const uint64_t t0 = globaltimer();
@@ -170,7 +165,7 @@ __device__ __forceinline__ void zero_slice(float *buf, size_t n, int c, int ncta
 // shared-memory state
 
 struct Smem {
-  uint8_t *ring, *op;
+  uint8_t *ring, *op, *stg;
   float *tbl;
   uint64_t *full, *empty, *opf, *stgb, *acc_ready, *drain, *att, *tblb;
   uint32_t *tmem_slot;
@@ -190,41 +185,46 @@ __device__ __forceinline__ uint4 *op_chunk(uint8_t *op, int j, int r, int cc) {
 }
 
 // Builds the bf16 operand of one GEMM unit from fp32 tiles staged by TMA and releases each
-// 64-wide K block to the MMA as soon as it is complete.  The unit's whole fp32 K slice (at most
-// 128 KB) is requested at once, so every box is in flight together: QKV / GU as 3-D boxes of
-// two K blocks of h (four 64-row x 32-column tiles); DN as two boxes per K block (the two gate
-// tiles, the two matching up tiles).  Each K block is converted in place: every thread first
-// reads its values of the block into registers, a barrier, then the bf16 block is written over
-// the first 8 KB of the block's own staging (the MMA descriptors point there).
+// 64-wide K block to the MMA as soon as it is complete.  Staging runs in groups of four
+// 64-row x 32-column tiles, double-buffered: QKV / GU fetch a group as one 3-D box of four
+// consecutive column tiles of h; DN as two boxes (two gate tiles, the two matching up tiles).
+// One wait, one proxy fence and one barrier per group; the group after next is issued as soon
+// as a buffer is consumed.
 //   QKV / GU:  bf16(h * (1 + scale)); designated units add the slice's sum of squares of h
 //   DN:        bf16(GELU_tanh(r*g + bg) * (r*u + bu)) from the gate/up accumulator
 __device__ void build_operand(const PersistParams &p, const Smem &sm, const CUtensorMap *tm_lh,
                               const CUtensorMap *tm_lg, int kind, int kb0, int nkb, const float *s1p,
-                              const float *bias, float *ss, bool stats, int M, uint32_t &stg_par, uint32_t &ntbl,
+                              const float *bias, float *ss, bool stats, int M, uint32_t &g, uint32_t &ntbl,
                               int tid) {
   const bool dn = kind == DN;
-  const int sb = slot_bytes(kind);
+  const int npieces = 2 * nkb;          // 32-column pieces of the unit's K slice
+  const int ppg = dn ? 2 : 4;           // pieces per group
+  const int ngroups = (npieces + ppg - 1) / ppg;
+  const uint32_t g0 = g;
   const int ncol = nkb * 64;            // table slice: scale (QKV, GU) or gate | up bias (DN)
-  if (tid == 0) {
-    const uint64_t pol = policy_evict_last();
+  uint64_t pol = 0;
+  // group q covers pieces [q * ppg, q * ppg + ppg) (a short last group reads its box's spare
+  // tiles from the neighbouring columns, or zero fill past the end; they are never used)
+  auto issue = [&](int q) {
+    const int buf = (g0 + q) % NGRP;
+    uint8_t *dst = sm.stg + buf * GRPB;
+    const int z = (kb0 * 64) / 32 + q * ppg;
+    mbar_arrive_expect_tx(&sm.stgb[buf], GRPB);
     if (dn) {
-      for (int j = 0; j < nkb; ++j) {
-        uint8_t *dst = sm.op + j * sb;
-        const int z = ((kb0 + j) * 64) / 32;
-        mbar_arrive_expect_tx(&sm.stgb[j], 4 * STG);
-        tma_load_3d(dst, tm_lg, &sm.stgb[j], 0, 0, z, pol);
-        tma_load_3d(dst + 2 * STG, tm_lg, &sm.stgb[j], 0, 0, z + F / 32, pol);
-      }
+      tma_load_3d(dst, tm_lg, &sm.stgb[buf], 0, 0, z, pol);
+      tma_load_3d(dst + 2 * STG, tm_lg, &sm.stgb[buf], 0, 0, z + F / 32, pol);
+    } else {
+      tma_load_3d(dst, tm_lh, &sm.stgb[buf], 0, 0, z, pol);
+    }
+  };
+  if (tid == 0) {
+    pol = policy_evict_last();
+    for (int q = 0; q < ngroups && q < NGRP; ++q) issue(q);
+    if (dn) {
       mbar_arrive_expect_tx(sm.tblb, 2 * ncol * 4);
       bulk_load(sm.tbl, bias + kb0 * 64, ncol * 4, sm.tblb);
       bulk_load(sm.tbl + ncol, bias + F + kb0 * 64, ncol * 4, sm.tblb);
     } else {
-      // a box of two K blocks; past the end of h (an odd slice at the last block) the box is
-      // zero-filled and that block is never used
-      for (int b = 0; 2 * b < nkb; ++b) {
-        mbar_arrive_expect_tx(&sm.stgb[b], 4 * STG);
-        tma_load_3d(sm.op + 2 * b * sb, tm_lh, &sm.stgb[b], 0, 0, (kb0 * 64) / 32 + 4 * b, pol);
-      }
       mbar_arrive_expect_tx(sm.tblb, ncol * 4);
       bulk_load(sm.tbl, s1p + kb0 * 64, ncol * 4, sm.tblb);
     }
@@ -235,24 +235,21 @@ __device__ void build_operand(const PersistParams &p, const Smem &sm, const CUte
   if (dn && r < M) rr = rsqrtf(__ldcg(ss + r) * (1.0f / D) + p.eps);
   wait_bar(sm.tblb, ntbl & 1, p.ctl, 642);
   ++ntbl;
-  for (int j = 0; j < nkb; ++j) {
-    uint8_t *slot = sm.op + j * sb;
-    const int bi = dn ? j : (j >> 1);
-    if (dn || (j & 1) == 0) {
-      wait_bar(&sm.stgb[bi], (stg_par >> bi) & 1, p.ctl, 641);
-      stg_par ^= 1u << bi;
-    }
-    uint4 out[2];
-#pragma unroll
-    for (int pc = 0; pc < 2; ++pc) {
-      const int col = j * 64 + pc * 32 + sub * 8;  // column within the unit's K slice
-      out[pc] = make_uint4(0, 0, 0, 0);
+  for (int q = 0; q < ngroups; ++q) {
+    const uint32_t gq = g0 + q;
+    const uint8_t *grp = sm.stg + (gq % NGRP) * GRPB;
+    wait_bar(&sm.stgb[gq % NGRP], (gq / NGRP) & 1, p.ctl, 641);
+    const int p0 = q * ppg, pe = p0 + ppg < npieces ? p0 + ppg : npieces;
+    for (int pc = p0; pc < pe; ++pc) {
+      const int col = pc * 32 + sub * 8;  // column within the unit's K slice
+      const int j = pc >> 1, cc = (pc & 1) * 4 + sub;
+      uint4 out = make_uint4(0, 0, 0, 0);
       if (r < M) {
         float v[8];
         if (dn) {
           float u[8];
-          stg_read8(slot + pc * STG, r, 2 * sub, v);
-          stg_read8(slot + (2 + pc) * STG, r, 2 * sub, u);
+          stg_read8(grp + (pc - p0) * STG, r, 2 * sub, v);
+          stg_read8(grp + (2 + pc - p0) * STG, r, 2 * sub, u);
           const float4 bg0 = *reinterpret_cast<const float4 *>(sm.tbl + col);
           const float4 bg1 = *reinterpret_cast<const float4 *>(sm.tbl + col + 4);
           const float4 bu0 = *reinterpret_cast<const float4 *>(sm.tbl + ncol + col);
@@ -262,7 +259,7 @@ __device__ void build_operand(const PersistParams &p, const Smem &sm, const CUte
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = gelu_tanh_fast(rr * v[e] + bgv[e]) * (rr * u[e] + buv[e]);
         } else {
-          stg_read8(slot + pc * STG, r, 2 * sub, v);
+          stg_read8(grp + (pc - p0) * STG, r, 2 * sub, v);
           const float4 s0 = *reinterpret_cast<const float4 *>(sm.tbl + col);
           const float4 s1 = *reinterpret_cast<const float4 *>(sm.tbl + col + 4);
           const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
@@ -272,20 +269,21 @@ __device__ void build_operand(const PersistParams &p, const Smem &sm, const CUte
             v[e] *= sv[e];
           }
         }
-        out[pc].x = pack_bf16(v[0], v[1]);
-        out[pc].y = pack_bf16(v[2], v[3]);
-        out[pc].z = pack_bf16(v[4], v[5]);
-        out[pc].w = pack_bf16(v[6], v[7]);
+        out.x = pack_bf16(v[0], v[1]);
+        out.y = pack_bf16(v[2], v[3]);
+        out.z = pack_bf16(v[4], v[5]);
+        out.w = pack_bf16(v[6], v[7]);
       }
+      *op_chunk(sm.op, j, r, cc) = out;
     }
-    named_sync();  // every read of this block's staging is done; block j - 1 is written
-    if (tid == 0 && j > 0) mbar_arrive(&sm.opf[j - 1]);
-#pragma unroll
-    for (int pc = 0; pc < 2; ++pc) *op_chunk(slot, 0, r, pc * 4 + sub) = out[pc];
-    fence_proxy_async_shared();  // this thread's part of block j: visible to the MMA
+    fence_proxy_async_shared();  // the group's K blocks are complete: visible to the MMA
+    named_sync();
+    if (tid == 0) {
+      for (int j = p0 >> 1; j < (pe >> 1); ++j) mbar_arrive(&sm.opf[j]);
+      if (q + NGRP < ngroups) issue(q + NGRP);  // refill the buffer just consumed
+    }
   }
-  named_sync();
-  if (tid == 0) mbar_arrive(&sm.opf[nkb - 1]);
+  g = g0 + ngroups;
   if (stats) {
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
@@ -295,9 +293,9 @@ __device__ void build_operand(const PersistParams &p, const Smem &sm, const CUte
 
 // ---------------------------------------------------------------------------------------
 // Q/K/V finalise: y = r * acc + bias, RoPE at position lv + q on the 8 query heads and the
-// key; bf16 Q [64][2048], K_s / V_s [64][256].  Eight (row, head) tasks per CTA, 32 threads
-// each (4 rotation pairs or 8 V columns per thread), so that C * 10 <= 8 * grid tasks take
-// one pass with every load of a thread in flight at once.
+// key; bf16 Q [64][2048], K_s / V_s [64][256].  Four (row, head) tasks per pass, 64 threads
+// each, every load of a pass in flight at once.
+
 __device__ void qkv_finalise(const PersistParams &p, int lv, size_t kl, int c, int ncta, int C, int tid) {
   const float *bias = p.bias_qkv + kl * 2560;
   const int lt = tid & 31;
@@ -506,7 +504,7 @@ __device__ void attn_unit(const PersistParams &p, const Smem &sm, const AttnCtx 
 }
 
 // Merges the key splits of rows (head, query) into the bf16 attention output.  Four rows at a
-// time, 64 threads x 4 dims per row; every split's partial of a thread is loaded at once.
+// time, 64 threads x 4 dims per row; the splits' partials are loaded in two halves.
 __device__ void combine_rows(const PersistParams &p, int nsplit, int c, int ncta, int C, int tid) {
   const int sub = tid >> 6, d0 = (tid & 63) * 4;
   for (int base = c * 4; base < NH * C; base += ncta * 4) {
@@ -574,50 +572,6 @@ __device__ void prefetch_tables(const PersistParams &p, int gp, int c, int ncta)
   }
 }
 
-// Cursor over this CTA's weight tiles of the whole loop, in the order the producer loads
-// them: steps, layers, GEMM kinds, this CTA's units, K blocks.
-struct TileCursor {
-  int S, L, c, ncta;
-  int k = 0, l = 0, kind = 0, u = 0, nt = 0, kb = 0, kb1 = 0;
-  bool ok = true;
-  __device__ TileCursor(const PersistParams &p, int c_, int ncta_) : S(p.S), L(p.L), c(c_), ncta(ncta_) {
-    u = first_unit(0, c, ncta);
-    settle();
-  }
-  // the first unit at or after (phase, u) that exists
-  __device__ void settle() {
-#pragma unroll 1
-    while (k < S) {
-      if (u < units(kind)) {
-        int kb0;
-        unit_kb(kind, u, nt, kb0, kb1);
-        kb = kb0;
-        return;
-      }
-      if (++kind == 4) {
-        kind = 0;
-        if (++l == L) {
-          l = 0;
-          ++k;
-        }
-      }
-      u = first_unit((k * L + l) * 4 + kind, c, ncta);
-    }
-    ok = false;
-  }
-  __device__ bool valid() const { return ok; }
-  __device__ void next() {
-    if (++kb < kb1) return;
-    u += ncta;
-    settle();
-  }
-  __device__ void prefetch(const CUtensorMap &mq, const CUtensorMap &mo, const CUtensorMap &mg,
-                           const CUtensorMap &md) const {
-    const CUtensorMap *map = kind == QKV ? &mq : (kind == OPJ ? &mo : (kind == GU ? &mg : &md));
-    tma_prefetch_l2_2d(map, kb * 64, l * rows_per_layer(kind) + nt * 128);
-  }
-};
-
 // ---------------------------------------------------------------------------------------
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -634,13 +588,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   Smem sm;
   sm.ring = smem;
   sm.op = smem + RING * WST;
-  sm.tbl = reinterpret_cast<float *>(sm.op + STAGE);
+  sm.stg = sm.op + OPB;
+  sm.tbl = reinterpret_cast<float *>(sm.stg + NGRP * GRPB);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm.op + REGION);
   sm.full = bars;
   sm.empty = bars + RING;
   sm.opf = bars + 2 * RING;
   sm.stgb = sm.opf + NOPK;
-  sm.acc_ready = sm.stgb + NSTB;
+  sm.acc_ready = sm.stgb + NGRP;
   sm.drain = sm.acc_ready + 1;
   sm.att = sm.drain + 1;
   sm.tblb = sm.att + 1;
@@ -674,11 +629,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint64_t pol = policy_evict_first();
       uint32_t it = 0;
       bool ok = true;
-      // L2 run-ahead: a second cursor over the same tile list, PREFETCH tiles ahead of the
-      // ring, so that HBM keeps streaming weights while the compute warps are in phases that
-      // consume none (attention, row work, barriers); the ring loads then hit L2
-      TileCursor pf(p, c, ncta);
-      for (int i = 0; i < PREFETCH && pf.valid(); ++i, pf.next()) pf.prefetch(tm_qkv, tm_o, tm_gu, tm_d);
       for (int k = 0; k < S && ok; ++k)
         for (int l = 0; l < L && ok; ++l)
           for (int kind = 0; kind < 4 && ok; ++kind) {
@@ -698,10 +648,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_arrive_expect_tx(&sm.full[slot], WST);
                 tma_load_2d(sm.ring + slot * WST, map, &sm.full[slot], kb * 64, l * rows_per_layer(kind) + nt * 128,
                             pol);
-                if (pf.valid()) {
-                  pf.prefetch(tm_qkv, tm_o, tm_gu, tm_d);
-                  pf.next();
-                }
               }
             }
           }
@@ -737,7 +683,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t a = smem_u32(sm.ring + slot * WST);
-                const uint32_t b = opb + j * slot_bytes(kind);
+                const uint32_t b = opb + j * 8192;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                   umma_bf16(tmem, sdesc_k128(a + 32 * q), sdesc_k128(b + 32 * q), idesc,
@@ -756,7 +702,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int cw = warp - 2;
     const int C = p.C, M = p.C;
     unsigned epoch = 0;
-    uint32_t nunit = 0, stg_par = 0, natt = 0, ntbl = 0;
+    uint32_t nunit = 0, gstg = 0, natt = 0, ntbl = 0;
     const CallArgs *ca = p.ca;
     AttnCtx ac;
     ac.lv = ca->valid_len[0];
@@ -834,18 +780,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint64_t pol = policy_evict_last();
                 for (int j = 0; j < nkb; ++j) {
                   mbar_arrive_expect_tx(&sm.opf[j], 8192);
-                  tma_load_2d(sm.op + j * slot_bytes(OPJ), &tm_lo, &sm.opf[j], (kb0 + j) * 64, 0, pol);
+                  tma_load_2d(sm.op + j * 8192, &tm_lo, &sm.opf[j], (kb0 + j) * 64, 0, pol);
                 }
               }
             } else if (kind == QKV) {
               build_operand(p, sm, &tm_lh, &tm_lg, kind, kb0, nkb, p.s1p_attn + kl * D, nullptr, p.ss_attn, nt == 0,
-                            M, stg_par, ntbl, tid);
+                            M, gstg, ntbl, tid);
             } else if (kind == GU) {
               build_operand(p, sm, &tm_lh, &tm_lg, kind, kb0, nkb, p.s1p_ffn + kl * D, nullptr, p.ss_ffn, nt == 0, M,
-                            stg_par, ntbl, tid);
+                            gstg, ntbl, tid);
             } else {
               build_operand(p, sm, &tm_lh, &tm_lg, kind, kb0, nkb, nullptr, p.bias_gu + kl * 2 * F, p.ss_ffn, false,
-                            M, stg_par, ntbl, tid);
+                            M, gstg, ntbl, tid);
             }
             if (tid == 0) stamp(p, epoch, 1);
             // epilogue: TMEM -> registers (x gate) -> shared tile [64 tokens][128 features] ->
