@@ -35,6 +35,13 @@ struct XMaps {
 int gemm_tile_index(int tn);
 GemmPlan gemm_plan(int M, int N, int K, int sm_count);
 cudaError_t gemm_init_attributes();
+// The 2-CTA form (gemm_tc2.cu): 256 weight rows x 256 tokens per SM pair.  Init records how
+// many 2-CTA clusters fit at once (0 disables the form); with RTVLA_PAIR_GEMM=1 set at init,
+// gemm_launch picks it for token tiles of 256 when N is a multiple of 256.
+cudaError_t gemm2_init_attributes(int sm_count);
+int gemm2_clusters();
+cudaError_t gemm2_launch(const CUtensorMap &tmW, const CUtensorMap &tmX128, const CUtensorMap &tmO,
+                         const GemmParams &p, cudaStream_t st);
 
 // out[m][n] (+)= col_scale[n] * sum_k X[m][k] W[w_row0 + n][k].  `accumulate` adds into the
 // existing contents of out; otherwise out must be zero when the plan splits K.

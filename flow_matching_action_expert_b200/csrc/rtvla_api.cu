@@ -664,7 +664,9 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
   if (cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess)
     return RTVLA_ERR_CUDA;
   if (!get_encoder()) return RTVLA_ERR_CUDA;
-  if (gemm_init_attributes() != cudaSuccess || attn_init_attributes() != cudaSuccess) return RTVLA_ERR_CUDA;
+  if (gemm_init_attributes() != cudaSuccess || attn_init_attributes() != cudaSuccess ||
+      gemm2_init_attributes(c->sm_count) != cudaSuccess)
+    return RTVLA_ERR_CUDA;
   if (cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking) != cudaSuccess) return RTVLA_ERR_CUDA;
 
   // ---- weights: Q|K|V stacked, gate|up stacked, layers stacked (one tensor map each)
