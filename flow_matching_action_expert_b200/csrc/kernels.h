@@ -72,7 +72,11 @@ struct AttnParams {
 
 cudaError_t attn_init_attributes();
 int attn_splits(int batch, int nq, int max_keys, int sm_count, int *keys_per_split);
+// Keys the split plan must cover: prefix and suffix are chunked separately (64 keys each).
+int attn_keys(int prefix_cap, int n_suf);
 cudaError_t attn_launch(const AttnParams &p, int batch, cudaStream_t st);
+cudaError_t attn_tc_init_attributes();
+cudaError_t attn_tc_launch(const AttnParams &p, int batch, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------
 // element-wise / row kernels

@@ -266,7 +266,7 @@ cudaError_t enqueue_denoise(rtvla_ctx *c, const CallArgs *dargs, int B, int cap,
   ap.vsuf = c->vs;
   ap.n_suf = C;
   ap.nq = C;
-  ap.n_splits = attn_splits(B, C, cap + C, c->sm_count, &ap.keys_per_split);
+  ap.n_splits = attn_splits(B, C, attn_keys(cap, C), c->sm_count, &ap.keys_per_split);
   ap.opart = c->opart;
   ap.mlpart = c->mlpart;
   ap.out = c->o;
@@ -331,7 +331,7 @@ cudaError_t enqueue_prefill(rtvla_ctx *c, const CallArgs *dargs, int B, int P, c
   ap.ca = dargs;
   ap.n_suf = 0;
   ap.nq = P;
-  ap.n_splits = attn_splits(B, P, P, c->sm_count, &ap.keys_per_split);
+  ap.n_splits = attn_splits(B, P, attn_keys(P, 0), c->sm_count, &ap.keys_per_split);
   ap.opart = c->popart;
   ap.mlpart = c->pmlpart;
   ap.out = c->po;
@@ -775,7 +775,7 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
   c->vs = dalloc<bf16>(c, M * HD);
   c->o = dalloc<bf16>(c, M * NQH * HD);
   c->mb = dalloc<bf16>(c, M * F);
-  const size_t parts = max_attn_partials(c->Bmax, C, c->Pmax + C, c->sm_count);
+  const size_t parts = max_attn_partials(c->Bmax, C, attn_keys(c->Pmax, C), c->sm_count);
   c->opart = dalloc<float>(c, parts * NQH * HD);
   c->mlpart = dalloc<float>(c, parts * NQH * 2);
   if (!c->x || !c->h || !c->r || !c->acc_qkv || !c->acc_gu || !c->op || !c->q || !c->ks || !c->vs || !c->o ||
@@ -790,7 +790,7 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
     c->pq = dalloc<bf16>(c, Mp * NQH * HD);
     c->po = dalloc<bf16>(c, Mp * NQH * HD);
     c->pmb = dalloc<bf16>(c, Mp * FP);
-    const size_t pparts = max_attn_partials(c->Bmax, c->Pmax, c->Pmax, c->sm_count);
+    const size_t pparts = max_attn_partials(c->Bmax, c->Pmax, attn_keys(c->Pmax, 0), c->sm_count);
     c->popart = dalloc<float>(c, pparts * NQH * HD);
     c->pmlpart = dalloc<float>(c, pparts * NQH * 2);
     if (!c->px || !c->pacc || !c->pop || !c->pq || !c->po || !c->pmb || !c->popart || !c->pmlpart)
