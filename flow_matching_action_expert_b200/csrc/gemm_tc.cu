@@ -112,7 +112,14 @@ __global__ void __launch_bounds__(192, 1)
           }
           uint8_t *st = smem + s * G::STAGE;
           mbar_arrive_expect_tx(&full[s], G::STAGE);
-          tma_load_2d(st, &tmW, &full[s], (ti.kb0 + i) * 64, p.w_row0 + ti.n0, pol_w);
+          if (p.glu) {
+            // gate rows f0 .. f0 + 63 over A rows 0..63, the matching up rows over A rows 64..127
+            const int f0 = ti.n0 >> 1;
+            tma_load_2d(st, &tmW, &full[s], (ti.kb0 + i) * 64, p.w_row0 + f0, pol_w);
+            tma_load_2d(st + G::W_BYTES / 2, &tmW, &full[s], (ti.kb0 + i) * 64, p.w_row0 + (p.N >> 1) + f0, pol_w);
+          } else {
+            tma_load_2d(st, &tmW, &full[s], (ti.kb0 + i) * 64, p.w_row0 + ti.n0, pol_w);
+          }
           tma_load_2d(st + G::W_BYTES, &tmX, &full[s], (ti.kb0 + i) * 64, ti.m0, pol_x);
         }
       }
@@ -185,14 +192,46 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) box[(c - c0 + j) * 128 + nl] = (ti.m0 + c + j < p.M) ? v[j] * sc : 0.f;
         }
-        fence_proxy_async_shared();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (leader) {
-          if (p.atomic)
-            tma_reduce_add_2d(&tmO, box, ti.n0, ti.m0 + c0);
-          else
-            tma_store_2d(&tmO, box, ti.n0, ti.m0 + c0);
-          bulk_commit();
+        if (p.glu) {
+          // box columns 0..63 hold the gate features, 64..127 the up features: thread t takes
+          // feature t % 64 for 32 of the 64 tokens, then the bf16 results replace the box as
+          // [64 tokens][64 features] with 128-byte swizzle, stored by one TMA copy
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          const int t = (warp - 2) * 32 + lane;
+          const int f = t & 63, th = t >> 6;
+          const int f0 = ti.n0 >> 1;
+          const float bg = p.glu_bias ? p.glu_bias[f0 + f] : 0.f;
+          const float bu = p.glu_bias ? p.glu_bias[(p.N >> 1) + f0 + f] : 0.f;
+          float mv[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tok = th * 32 + j, row = ti.m0 + c0 + tok;
+            const float rr = (p.glu_r != nullptr && row < p.M) ? p.glu_r[row] : 1.f;
+            mv[j] = gelu_tanh(rr * box[tok * 128 + f] + bg) * (rr * box[tok * 128 + 64 + f] + bu);
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");  // every read of the fp32 box is done
+          bf16 *ob = reinterpret_cast<bf16 *>(box);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tok = th * 32 + j;
+            ob[tok * 64 + ((((f >> 3) ^ (tok & 7)) << 3) | (f & 7))] = f2bf(mv[j]);
+          }
+          fence_proxy_async_shared();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (leader) {
+            tma_store_2d(&tmO, box, f0, ti.m0 + c0);
+            bulk_commit();
+          }
+        } else {
+          fence_proxy_async_shared();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (leader) {
+            if (p.atomic)
+              tma_reduce_add_2d(&tmO, box, ti.n0, ti.m0 + c0);
+            else
+              tma_store_2d(&tmO, box, ti.n0, ti.m0 + c0);
+            bulk_commit();
+          }
         }
       }
       // the accumulator has been read: hand it back to the MMA issuer
@@ -232,6 +271,20 @@ cudaError_t gemm_init_attributes() {
   return e;
 }
 
+static cudaError_t launch_plan(const CUtensorMap &tmW, const XMaps &xm, const CUtensorMap &tmO, int tn,
+                               const GemmParams &p, int sm_count, cudaStream_t st) {
+  const CUtensorMap &tmX = xm.m[gemm_tile_index(tn)];
+  switch (tn) {
+    case 64: return launch_tn<64>(tmW, tmX, tmO, p, sm_count, st);
+    case 128: return launch_tn<128>(tmW, tmX, tmO, p, sm_count, st);
+    default:
+      // several tiles per CTA, or a long K slice: the deeper ring
+      if (p.m_tiles * p.n_tiles * p.splits > sm_count || p.kb_per_split >= 32)
+        return launch_tn<256, true>(tmW, tmX, tmO, p, sm_count, st);
+      return launch_tn<256>(tmW, tmX, tmO, p, sm_count, st);
+  }
+}
+
 // Chooses the token tile and the K split (at most one round of tiles over the SMs).
 GemmPlan gemm_plan(int M, int N, int K, int sm_count) {
   GemmPlan g;
@@ -259,7 +312,7 @@ cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int
                         int sm_count, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   GemmPlan g = gemm_plan(M, N, K, sm_count);
-  GemmParams p;
+  GemmParams p{};
   p.M = M;
   p.N = N;
   p.K = K;
@@ -287,16 +340,32 @@ cudaError_t gemm_launch(const CUtensorMap &tmW, int w_row0, const XMaps &xm, int
     p.atomic = (accumulate || p.splits > 1) ? 1 : 0;
     return gemm2_launch(tmW, xm.m[1], tmO, p, st);
   }
-  const CUtensorMap &tmX = xm.m[gemm_tile_index(g.tn)];
-  switch (g.tn) {
-    case 64: return launch_tn<64>(tmW, tmX, tmO, p, sm_count, st);
-    case 128: return launch_tn<128>(tmW, tmX, tmO, p, sm_count, st);
-    default:
-      // several tiles per CTA, or a long K slice: the deeper ring
-      if (p.m_tiles * p.n_tiles * p.splits > sm_count || p.kb_per_split >= 32)
-        return launch_tn<256, true>(tmW, tmX, tmO, p, sm_count, st);
-      return launch_tn<256>(tmW, tmX, tmO, p, sm_count, st);
-  }
+  return launch_plan(tmW, xm, tmO, g.tn, p, sm_count, st);
+}
+
+bool gemm_glu_applies(int M, int F, int K, int sm_count) { return gemm_plan(M, 2 * F, K, sm_count).splits == 1; }
+
+cudaError_t gemm_launch_glu(const CUtensorMap &tmW64, int w_row0, const XMaps &xm, int M, int F, int K,
+                            const CUtensorMap &tmM, const float *r, const float *bias, DevCtl *ctl, int sm_count,
+                            cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  const GemmPlan g = gemm_plan(M, 2 * F, K, sm_count);
+  if (g.splits != 1) return cudaErrorInvalidValue;
+  GemmParams p{};
+  p.M = M;
+  p.N = 2 * F;
+  p.K = K;
+  p.w_row0 = w_row0;
+  p.kb_per_split = g.kb_per_split;
+  p.ldo = F;
+  p.ctl = ctl;
+  p.m_tiles = g.m_tiles;
+  p.n_tiles = g.n_tiles;
+  p.splits = 1;
+  p.glu = 1;
+  p.glu_r = r;
+  p.glu_bias = bias;
+  return launch_plan(tmW64, xm, tmM, g.tn, p, sm_count, st);
 }
 
 }  // namespace rtvla

@@ -21,6 +21,13 @@ struct GemmParams {
   int atomic;              // 1: fp32 reduction into out; 0: plain store
   DevCtl *ctl;
   int m_tiles, n_tiles, splits;  // the launch's tiles (a CTA loops over tile c, c + grid, ...)
+  // gated-GELU epilogue (glu = 1): the weight is [gate rows ; up rows] (N = 2F); tile n holds
+  // gate rows n*64 .. n*64+63 and the matching up rows, and the epilogue writes
+  // bf16 GELU_tanh(r*g + b_g) * (r*u + b_u) for features n*64 .. n*64+63 (r per token row,
+  // b from glu_bias [2F]; either may be null) through a bf16 map of the [M][F] output
+  int glu;
+  const float *glu_r;
+  const float *glu_bias;
 };
 
 struct GemmPlan {
@@ -42,6 +49,15 @@ cudaError_t gemm2_init_attributes(int sm_count);
 int gemm2_clusters();
 cudaError_t gemm2_launch(const CUtensorMap &tmW, const CUtensorMap &tmX128, const CUtensorMap &tmO,
                          const GemmParams &p, cudaStream_t st);
+
+// Gated-GELU form of gemm_launch: m[t][f] = GELU_tanh(r[t] g + b_g[f]) * (r[t] u + b_u[f]) with
+// g, u = X W^T over the gate rows w_row0 + f and the up rows w_row0 + F + f of tmW64 (a map
+// with 64-row boxes); written as bf16 through tmM (64 x 64 boxes, 128-byte swizzle).  Needs
+// the whole K in one tile: returns false (nothing launched) when the plan would split K.
+bool gemm_glu_applies(int M, int F, int K, int sm_count);
+cudaError_t gemm_launch_glu(const CUtensorMap &tmW64, int w_row0, const XMaps &xm, int M, int F, int K,
+                            const CUtensorMap &tmM, const float *r, const float *bias, DevCtl *ctl, int sm_count,
+                            cudaStream_t st);
 
 // out[m][n] (+)= col_scale[n] * sum_k X[m][k] W[w_row0 + n][k].  `accumulate` adds into the
 // existing contents of out; otherwise out must be zero when the plan splits K.

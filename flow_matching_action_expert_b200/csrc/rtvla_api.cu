@@ -75,6 +75,7 @@ struct rtvla_ctx {
   DevCtl *ctl = nullptr;
   CallArgs *args_dn = nullptr, *args_pf = nullptr, *args_tr = nullptr;
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_pwqkv, tm_pwo, tm_pwgu, tm_pwd;
+  CUtensorMap tm_wgu64, tm_pwgu64;  // the gate/up weights with 64-row boxes (gated-GELU GEMM)
   // fp32 GEMM outputs of the layered engine, 128-column x 64-row boxes (bulk store / reduce-add)
   CUtensorMap tmo_qkv, tmo_h, tmo_gu, tmo_pqkv, tmo_px, tmo_pgu;
   PersistMaps pmaps;                // tensor maps of the persistent engine
@@ -255,7 +256,10 @@ cudaError_t enqueue_denoise(rtvla_ctx *c, const CallArgs *dargs, int B, int cap,
   const int L = c->L, S = c->S, C = c->C, M = B * C;
   const float eps = c->cfg.rms_eps;
   CKR(cudaMemsetAsync(c->acc_qkv, 0, (size_t)M * 2560 * 4, st));
-  CKR(cudaMemsetAsync(c->acc_gu, 0, (size_t)M * 2 * F * 4, st));
+  // the gate/up GEMM writes GELU(g) * u directly when its plan keeps K whole; otherwise it
+  // accumulates into acc_gu (zeroed here; k_gelu_mul re-zeroes what it consumed)
+  const bool glu = gemm_glu_applies(M, F, D, c->sm_count);
+  if (!glu) CKR(cudaMemsetAsync(c->acc_gu, 0, (size_t)M * 2 * F * 4, st));
   CKN(launch_init_x(dargs, c->x, M * A, C, c->first, st));
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
@@ -297,9 +301,14 @@ cudaError_t enqueue_denoise(rtvla_ctx *c, const CallArgs *dargs, int B, int cap,
       CKN(gemm_launch(c->tm_wo, l * D, c->tm_o, M, D, NQH * HD, c->h, c->tmo_h, D, c->gate_attn + kl * D, true, c->ctl,
                       c->sm_count, st));
       CKN(launch_adanorm(c->h, c->s1p_ffn + kl * D, c->op, c->r, M, eps, st));
-      CKN(gemm_launch(c->tm_wgu, l * 2 * F, c->tm_op, M, 2 * F, D, c->acc_gu, c->tmo_gu, 2 * F, nullptr, false, c->ctl,
-                      c->sm_count, st));
-      CKN(launch_gelu_mul(c->acc_gu, c->r, c->bias_gu + kl * 2 * F, c->mb, M, F, st));
+      if (glu) {
+        CKN(gemm_launch_glu(c->tm_wgu64, l * 2 * F, c->tm_op, M, F, D, c->tm_mb.m[0], c->r, c->bias_gu + kl * 2 * F,
+                            c->ctl, c->sm_count, st));
+      } else {
+        CKN(gemm_launch(c->tm_wgu, l * 2 * F, c->tm_op, M, 2 * F, D, c->acc_gu, c->tmo_gu, 2 * F, nullptr, false,
+                        c->ctl, c->sm_count, st));
+        CKN(launch_gelu_mul(c->acc_gu, c->r, c->bias_gu + kl * 2 * F, c->mb, M, F, st));
+      }
       CKN(gemm_launch(c->tm_wd, l * D, c->tm_mb, M, D, F, c->h, c->tmo_h, D, c->gate_ffn + kl * D, true, c->ctl,
                       c->sm_count, st));
       if (trace && k == last_step)
@@ -321,7 +330,10 @@ cudaError_t enqueue_prefill(rtvla_ctx *c, const CallArgs *dargs, int B, int P, c
   int n = 0;
   const int L = c->L, M = B * P;
   const float eps = c->cfg.rms_eps;
-  CKR(cudaMemsetAsync(c->pacc, 0, (size_t)M * 2 * FP * 4, st));
+  // the QKV accumulator (the first M x 2560 floats of pacc) must start at zero, and the
+  // gate/up accumulator too unless the gate/up GEMM writes GELU(g) * u directly
+  const bool glu = gemm_glu_applies(M, FP, DP, c->sm_count);
+  CKR(cudaMemsetAsync(c->pacc, 0, (size_t)M * (glu ? 2560 : 2 * FP) * 4, st));
   CKN(launch_pf_mask(dargs, B, P, c->ctl, st));
   CKN(launch_pf_embed(dargs, c->px, M, DP, st));
   AttnParams ap;
@@ -349,9 +361,14 @@ cudaError_t enqueue_prefill(rtvla_ctx *c, const CallArgs *dargs, int B, int P, c
     CKN(gemm_launch(c->tm_pwo, l * DP, c->tm_po, M, DP, NQH * HD, c->px, c->tmo_px, DP, nullptr, true, c->ctl,
                     c->sm_count, st));
     CKN(launch_rmsnorm(c->px, c->pop, M, DP, eps, st));
-    CKN(gemm_launch(c->tm_pwgu, l * 2 * FP, c->tm_pop, M, 2 * FP, DP, c->pacc, c->tmo_pgu, 2 * FP, nullptr, false, c->ctl,
-                    c->sm_count, st));
-    CKN(launch_gelu_mul(c->pacc, nullptr, nullptr, c->pmb, M, FP, st));
+    if (glu) {
+      CKN(gemm_launch_glu(c->tm_pwgu64, l * 2 * FP, c->tm_pop, M, FP, DP, c->tm_pmb.m[0], nullptr, nullptr, c->ctl,
+                          c->sm_count, st));
+    } else {
+      CKN(gemm_launch(c->tm_pwgu, l * 2 * FP, c->tm_pop, M, 2 * FP, DP, c->pacc, c->tmo_pgu, 2 * FP, nullptr, false,
+                      c->ctl, c->sm_count, st));
+      CKN(launch_gelu_mul(c->pacc, nullptr, nullptr, c->pmb, M, FP, st));
+    }
     CKN(gemm_launch(c->tm_pwd, l * DP, c->tm_pmb, M, DP, FP, c->px, c->tmo_px, DP, nullptr, true, c->ctl, c->sm_count, st));
   }
   *kernels = n;
@@ -805,6 +822,7 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
             make_map(&c->tm_wqkv, c->w_qkv, (uint64_t)L * 2560, D, 128) &&
             make_map(&c->tm_wo, c->w_o, (uint64_t)L * D, NQH * HD, 128) &&
             make_map(&c->tm_wgu, c->w_gu, (uint64_t)L * 2 * F, D, 128) &&
+            make_map(&c->tm_wgu64, c->w_gu, (uint64_t)L * 2 * F, D, 64) &&
             make_map(&c->tm_wd, c->w_d, (uint64_t)L * D, F, 128) && make_xmaps(&c->tm_op, c->op, M, D) &&
             make_xmaps(&c->tm_o, c->o, M, NQH * HD) && make_xmaps(&c->tm_mb, c->mb, M, F) &&
             make_map(&c->tm_q64, c->q, M, NQH * HD, 64) && make_map_f32(&c->tmo_qkv, c->acc_qkv, M, 2560, 128, false) &&
@@ -813,6 +831,7 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
     ok = ok && make_map(&c->tm_pwqkv, c->pw_qkv, (uint64_t)L * 2560, DP, 128) &&
          make_map(&c->tm_pwo, c->pw_o, (uint64_t)L * DP, NQH * HD, 128) &&
          make_map(&c->tm_pwgu, c->pw_gu, (uint64_t)L * 2 * FP, DP, 128) &&
+         make_map(&c->tm_pwgu64, c->pw_gu, (uint64_t)L * 2 * FP, DP, 64) &&
          make_map(&c->tm_pwd, c->pw_d, (uint64_t)L * DP, FP, 128) &&
          make_xmaps(&c->tm_pop, c->pop, Mp, DP) && make_xmaps(&c->tm_po, c->po, Mp, NQH * HD) &&
          make_xmaps(&c->tm_pmb, c->pmb, Mp, FP) && make_map_f32(&c->tmo_pqkv, c->pacc, Mp, 2560, 128, false) &&
