@@ -14,9 +14,9 @@
 //   O += P V      tcgen05.mma M = 128, N = 256 (head dim), K = 64 keys, P from shared memory
 //                 (K-major), V in its row-major [key][dim] layout as an MN-major operand
 // Warps 0-3: softmax and output (warp w reads TMEM lanes 32w..32w+31); warps 4-7: loaders
-// (16-byte cp.async copies into the 128-byte-swizzled operand layout, then a proxy fence); warp 8: TMEM
-// owner, lane 0 issues the MMAs.  Splits are merged by k_attn_combine.  Every wait is
-// bounded (DevCtl::timeout_ns).
+// (16-byte cp.async copies into the 128-byte-swizzled operand layout, then a proxy fence;
+// warps 4-5 stage K, 6-7 V); warp 8: TMEM owner, lane 0 issues the MMAs.  Splits are merged
+// by k_attn_combine.  Every wait is bounded (DevCtl::timeout_ns).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -29,7 +29,7 @@ constexpr int Q_BYTES = 4 * ROWS * 128;     // 4 column blocks of [128 rows][64 
 constexpr int KV_BYTES = 4 * KC * 128;      // 4 column blocks of [64 keys][64 bf16]
 constexpr int P_BYTES = ROWS * 128;         // [128 rows][64 keys] bf16
 constexpr int THREADS = 288;
-constexpr int NBAR = 13;
+constexpr int NBAR = 17;
 constexpr int SMEM = Q_BYTES + 4 * KV_BYTES + 2 * P_BYTES + 1024 + NBAR * 8 + 16;
 static_assert(SMEM <= 232448, "shared memory per CTA");
 constexpr float RESCALE_LOG2 = 8.f;
@@ -106,12 +106,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
   const uint32_t ks0 = qs + Q_BYTES, vs0 = qs + Q_BYTES + 2 * KV_BYTES, ps0 = qs + Q_BYTES + 4 * KV_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Q_BYTES + 4 * KV_BYTES + 2 * P_BYTES);
   uint64_t *q_full = bars;          // loaders -> MMA: Q staged
-  uint64_t *kv_full = bars + 1;     // [2] loaders -> MMA: K and V of a chunk staged
-  uint64_t *kv_empty = bars + 3;    // [2] MMA -> loaders: the chunk's S and PV MMAs are done
-  uint64_t *s_full = bars + 5;      // [2] MMA -> softmax: S in TMEM
-  uint64_t *s_empty = bars + 7;     // [2] softmax -> MMA: S read
-  uint64_t *p_full = bars + 9;      // [2] softmax -> MMA: P written (and O rescaled)
-  uint64_t *p_empty = p_full + 2;   // [2] MMA -> softmax: PV done (P buffer free, O current)
+  uint64_t *k_full = bars + 1;      // [2] K loaders -> MMA: a chunk's K staged
+  uint64_t *k_empty = bars + 3;     // [2] MMA -> K loaders: the chunk's S MMAs are done
+  uint64_t *v_full = bars + 5;      // [2] V loaders -> MMA: a chunk's V staged
+  uint64_t *v_empty = bars + 7;     // [2] MMA -> V loaders: the chunk's PV MMAs are done
+  uint64_t *s_full = bars + 9;      // [2] MMA -> softmax: S in TMEM
+  uint64_t *s_empty = bars + 11;    // [2] softmax -> MMA: S read
+  uint64_t *p_full = bars + 13;     // [2] softmax -> MMA: P written (and O rescaled)
+  uint64_t *p_empty = bars + 15;    // [2] MMA -> softmax: PV done (P buffer free, O current)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(p_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,8 +137,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
   if (threadIdx.x == 0) {
     mbar_init(q_full, 128);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 128);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 64);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 64);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 128);
       mbar_init(&p_full[i], 128);
@@ -157,7 +161,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
     // ------------------------------------------------------------------ loaders
     // 16-byte cp.async copies straight into the swizzled operand layout (zero-filled where a
     // key or query does not exist); each thread waits for its own copies, fences them to the
-    // async proxy and arrives.  Chunk i + 1 is requested while chunk i is being computed.
+    // async proxy and arrives.  Warps 4-5 stage K, warps 6-7 stage V, each on its own pair of
+    // buffers: K of chunk i + 2 is requested once S of chunk i is done, V once its PV is.
     const int lt = threadIdx.x - 128;
     // Q: 128 rows x 32 chunks of 16 bytes; rows of queries past nq are zero
 #pragma unroll 4
@@ -173,25 +178,29 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
     cp_async_wait_all();
     fence_proxy_async_shared();
     mbar_arrive(q_full);
+    const bool is_k = warp < 6;
+    const int gt = lt & 63;  // thread within the K or the V group
+    uint64_t *full = is_k ? k_full : v_full;
+    uint64_t *empty = is_k ? k_empty : v_empty;
 #pragma unroll 1
     for (int i = 0; i < nch; ++i) {
       const int bb = i & 1;
-      if (i >= 2 && !mbar_wait(&kv_empty[bb], ((i >> 1) & 1) ^ 1, p.ctl, 212)) break;
+      if (i >= 2 && !mbar_wait(&empty[bb], ((i >> 1) & 1) ^ 1, p.ctl, 212)) break;
       const Chunk ch = chunk_at(p, kpre, vpre, lv, npc, b, c_begin + i);
-      const uint32_t kd = ks0 + bb * KV_BYTES, vd = vs0 + bb * KV_BYTES;
-#pragma unroll 4
-      for (int m = 0; m < 16; ++m) {
-        const int idx = lt + 128 * m;
+      const uint32_t dst = (is_k ? ks0 : vs0) + bb * KV_BYTES;
+      const bf16 *src = is_k ? ch.k : ch.v;
+#pragma unroll 8
+      for (int m = 0; m < 32; ++m) {
+        const int idx = gt + 64 * m;
         const int j = idx >> 5, cc = idx & 31;
         const bool ok = j < ch.nvalid;
-        const size_t off = (size_t)(ok ? j : 0) * HD + cc * 8;
-        cp_async16(swz(kd + (cc >> 3) * (KC * 128), j, cc & 7), ch.k + off, ok ? 16u : 0u);
-        cp_async16(swz(vd + (cc >> 3) * (KC * 128), j, cc & 7), ch.v + off, ok ? 16u : 0u);
+        cp_async16(swz(dst + (cc >> 3) * (KC * 128), j, cc & 7), src + (size_t)(ok ? j : 0) * HD + cc * 8,
+                   ok ? 16u : 0u);
       }
       cp_async_commit();
       cp_async_wait_all();
       fence_proxy_async_shared();
-      mbar_arrive(&kv_full[bb]);
+      mbar_arrive(&full[bb]);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------------ MMA issuer
@@ -201,7 +210,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
       bool ok = mbar_wait(q_full, 0, p.ctl, 213);
       auto issue_s = [&](int i) -> bool {
         const int bb = i & 1;
-        if (!mbar_wait(&kv_full[bb], (i >> 1) & 1, p.ctl, 214)) return false;
+        if (!mbar_wait(&k_full[bb], (i >> 1) & 1, p.ctl, 214)) return false;
         if (i >= 2 && !mbar_wait(&s_empty[bb], ((i >> 1) & 1) ^ 1, p.ctl, 215)) return false;
         tc_fence_after();
         const uint32_t kb0 = ks0 + bb * KV_BYTES;
@@ -212,6 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
             umma_bf16(tmem + (uint32_t)(bb * KC), sdesc_k128(qs + kb * (ROWS * 128) + 32 * k),
                       sdesc_k128(kb0 + kb * (KC * 128) + 32 * k), idesc_s, (kb | k) ? 1u : 0u);
         umma_commit(&s_full[bb]);
+        umma_commit(&k_empty[bb]);
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -219,7 +229,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
       for (int i = 0; i < nch && ok; ++i) {
         if (i + 1 < nch && !issue_s(i + 1)) break;
         const int bb = i & 1;
-        if (!mbar_wait(&p_full[bb], (i >> 1) & 1, p.ctl, 216)) break;
+        if (!mbar_wait(&p_full[bb], (i >> 1) & 1, p.ctl, 216) || !mbar_wait(&v_full[bb], (i >> 1) & 1, p.ctl, 221))
+          break;
         tc_fence_after();
         const uint32_t pa = ps0 + bb * P_BYTES, va = vs0 + bb * KV_BYTES;
 #pragma unroll
@@ -227,7 +238,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_attn_tc(AttnParams p) {
           umma_bf16(tmem + 2 * KC, sdesc_k128(pa + 32 * k), sdesc_mn128(va + k * 16 * 128, KC * 128), idesc_pv,
                     (i > 0 || k > 0) ? 1u : 0u);
         umma_commit(&p_empty[bb]);
-        umma_commit(&kv_empty[bb]);
+        umma_commit(&v_empty[bb]);
       }
     }
   } else {

@@ -3,8 +3,9 @@
 Checked mode (RTVLA_CHECKED=1 at rtvla_create) places every library buffer between guard
 bands and verifies them in rtvla_sync_status; it stands in for an out-of-bounds / race
 detector.  The bands must survive every engine (persistent kernel, layered graph at batch 1
-and at a ragged batch) and the prefix pass, and a planted overwrite past the residual-stream
-buffer must be reported as RTVLA_ERR_GUARD_OVERWRITE, after which the context still works.
+and at a ragged batch, the batch-16 kernels: tcgen05 attention and the gated-GELU GEMM) and
+the prefix pass, and a planted overwrite past the residual-stream buffer must be reported
+as RTVLA_ERR_GUARD_OVERWRITE, after which the context still works.
 
 RTVLA_DEVICE_MEMORY_CAP caps the context's device memory: rtvla_create must then return
 RTVLA_ERR_OOM and free everything it had allocated.
@@ -55,6 +56,23 @@ def test_guard_bands_hold_on_every_engine_and_catch_a_planted_overwrite(monkeypa
     assert R.rtvla_sync_status(m.ctx) == 0
     out2 = m.sample(noise, k, v, valid)
     assert_actions_close(out2, O.sample_actions(wf, wl.expert, noise, kn, vn, vnp), "checked B2 after the plant")
+    m.close()
+
+
+def test_guard_bands_hold_on_the_batched_layered_kernels(monkeypatch):
+    # batch 16 x chunk 63: the tcgen05 attention (64 sample x query-block units) and the
+    # gated-GELU gate/up GEMM (K kept whole), over ragged lengths with garbage in the padding
+    monkeypatch.setenv("RTVLA_CHECKED", "1")
+    base = WL.workload(1)
+    lens = (0, 1, 7, 63, 64, 65, 127, 128, 129, 200, 13, 190, 64, 1, 0, 150)
+    wl = WL.Workload("checked L2 P200 C63 B16", base.expert, 63, 16, 200, lens)
+    bits = WL.expert_weights(wl.expert, stressed=True)
+    m = GpuModel(wl, bits)
+    k, v, valid, kf, vf, vnp = device_kv(wl, pad_fill=3.0e4)
+    noise = WL.noise(wl)
+    out = m.sample(noise, k, v, valid)
+    assert R.rtvla_sync_status(m.ctx) == 0
+    assert_actions_close(out, O.sample_actions(WL.as_f32(bits), wl.expert, noise, kf, vf, vnp), wl.name)
     m.close()
 
 
