@@ -251,7 +251,8 @@ int attn_splits(int batch, int nq, int max_keys, int sm_count, int *keys_per_spl
   const int qblocks = (nq + QB - 1) / QB;
   const int chunks = (max_keys + KC - 1) / KC;
   const int base = batch * qblocks;
-  int splits = (sm_count + base - 1) / base;
+  // as many splits as keep every CTA in one wave over the SMs
+  int splits = sm_count / base;
   if (splits > chunks) splits = chunks;
   if (splits < 1) splits = 1;
   const int cps = (chunks + splits - 1) / splits;
