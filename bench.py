@@ -445,8 +445,8 @@ def run_ours(args, rank, world, local_rank):
 def run_pi0(args, rank, world, local_rank, wl):
     """The 2-view workload on the pi0 suffix variant: the suffix is [state token ; 63 action
     tokens], the action tokens come from the folded action-time MLP, plain RMSNorm, ungated
-    residuals (layered engine).  e2e: pinned host noise, state and cache copied in, the call,
-    the actions copied out, all inside the timed region."""
+    residuals (the persistent kernel at batch 1 unless --engine 1).  e2e: pinned host noise,
+    state and cache copied in, the call, the actions copied out, all inside the timed region."""
     import torch
 
     import flow_matching_action_expert_b200 as R
@@ -530,9 +530,11 @@ def run_pi0(args, rank, world, local_rank, wl):
         "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) bf16 weights and biases, N(0,1) KV, noise, state)",
         "config": dict(workload_config(wl, world), workload="pi0 " + wl.name, suffix_tokens=wl.chunk + 1),
-        "engine": "layered", "l2": "flushed by a 256 MiB write between timed loops",
+        "engine": "persistent" if kernels == 1 else "layered",
+        "l2": "flushed by a 256 MiB write between timed loops",
         "roofline": {"bound": "hbm" if t_mem >= t_tc else "tensor",
-                     "kernel": "rtvla_sample_actions_pi0 (one graph replay)",
+                     "kernel": ("k_persistent (one launch = one call)" if kernels == 1
+                                else "rtvla_sample_actions_pi0 (one graph replay)"),
                      "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
                      "traffic": None, "peak_source": src, "algorithmic_bytes_per_launch": int(b_loop),
                      "algorithmic_flops_per_launch": int(f_loop), "roofline_ms": round(max(t_mem, t_tc) * 1e3, 4)},

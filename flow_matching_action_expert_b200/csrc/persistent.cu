@@ -574,6 +574,86 @@ __device__ void prefetch_tables(const PersistParams &p, int gp, int c, int ncta)
 
 // ---------------------------------------------------------------------------------------
 
+// π0 suffix, token row c (CTA c, 256 threads): row 0 (the state token) gets W_st s + b_st in h;
+// an action row gets the operand of the action-time output linear,
+// op[c] = bf16(SiLU(W_fold x + c_k)), x = this row's actions (xr, 32 floats in shared memory).
+// Thread t computes outputs t, t + 256, t + 512, t + 768, every weight load issued up front.
+__device__ void pi0_row_in(const PersistParams &p, int c, int k, const float *xr, int tid) {
+  float xv[A];
+#pragma unroll
+  for (int j = 0; j < A; ++j) xv[j] = xr[j];
+#pragma unroll 1
+  for (int e = 0; e < 4; ++e) {
+    const int n = tid + NCOMP * e;
+    if (c == 0) {
+      uint4 w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[q] = __ldg(reinterpret_cast<const uint4 *>(p.w_st + (size_t)n * A) + q);
+      float acc = __ldg(p.b_st + n);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bf16 *wb = reinterpret_cast<const bf16 *>(&w[q]);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc += bf2f(wb[t]) * xv[q * 8 + t];
+      }
+      p.h[n] = acc;
+    } else {
+      float4 w[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) w[q] = __ldg(reinterpret_cast<const float4 *>(p.w_fold + (size_t)n * A) + q);
+      float acc = __ldg(p.c_tab + (size_t)k * D + n);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        acc += w[q].x * xv[4 * q] + w[q].y * xv[4 * q + 1] + w[q].z * xv[4 * q + 2] + w[q].w * xv[4 * q + 3];
+      p.op_ato[(size_t)c * D + n] = f2bf(acc / (1.0f + __expf(-acc)));
+    }
+  }
+}
+
+// π0: h[r][n] = b_ato[n] + sum_j op[r][j] W_ato[n][j] for the action rows r = 1 .. M-1.  CTA
+// c < 64 takes output features 16c .. 16c + 15, two per warp.  The operand rows are staged in
+// shared memory with a 16-byte pad per row (so that the lanes' rows fall in different banks);
+// lane l accumulates rows 1 + l and 33 + l over the whole K, the weights read as broadcasts.
+constexpr int OPS_LD = D / 8 + 1;  // staged operand row stride, in 16-byte chunks
+__device__ void pi0_ato(const PersistParams &p, const Smem &sm, int c, int M, int tid) {
+  if (c >= D / 16) return;
+  uint4 *ops = reinterpret_cast<uint4 *>(sm.op);  // [64][OPS_LD] chunks of 8 bf16 (~129 KB)
+  for (int i = tid; i < M * (D / 8); i += NCOMP)
+    ops[(i >> 7) * OPS_LD + (i & 127)] = __ldcg(reinterpret_cast<const uint4 *>(p.op_ato) + i);
+  named_sync();
+  const int w = tid >> 5, lane = tid & 31;
+  const int n0 = c * 16 + w * 2;
+  const int ra = 1 + lane, rb = 33 + lane;
+  const bool va = ra < M, vb = rb < M;
+  const uint4 *oa = ops + (size_t)(va ? ra : 0) * OPS_LD, *ob = ops + (size_t)(vb ? rb : 0) * OPS_LD;
+  const uint4 *w0 = reinterpret_cast<const uint4 *>(p.w_ato + (size_t)n0 * D);
+  const uint4 *w1 = reinterpret_cast<const uint4 *>(p.w_ato + (size_t)(n0 + 1) * D);
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll 4
+  for (int q = 0; q < D / 8; ++q) {
+    const uint4 x0 = __ldg(w0 + q), x1 = __ldg(w1 + q), ya = oa[q], yb = ob[q];
+    const bf16 *e0 = reinterpret_cast<const bf16 *>(&x0), *e1 = reinterpret_cast<const bf16 *>(&x1);
+    const bf16 *fa = reinterpret_cast<const bf16 *>(&ya), *fb = reinterpret_cast<const bf16 *>(&yb);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const float u0 = bf2f(e0[t]), u1 = bf2f(e1[t]), ga = bf2f(fa[t]), gb = bf2f(fb[t]);
+      a0 += u0 * ga;
+      a1 += u1 * ga;
+      b0 += u0 * gb;
+      b1 += u1 * gb;
+    }
+  }
+  const float bias0 = __ldg(p.b_ato + n0), bias1 = __ldg(p.b_ato + n0 + 1);
+  if (va) {
+    p.h[(size_t)ra * D + n0] = a0 + bias0;
+    p.h[(size_t)ra * D + n0 + 1] = a1 + bias1;
+  }
+  if (vb) {
+    p.h[(size_t)rb * D + n0] = b0 + bias0;
+    p.h[(size_t)rb * D + n0 + 1] = b1 + bias1;
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     k_persistent(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_o,
                  const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CUtensorMap tm_d,
@@ -725,7 +805,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       p.qb[(size_t)C * 2048 + i] = f2bf(0.f);
     }
     float *xs = reinterpret_cast<float *>(sm.op);
-    if (c < M) {
+    if (p.pi0 && c < M) {
+      // π0: the state row, and the action rows' operands of the action-time output linear
+      if (tid < A) {
+        float v;
+        if (c == 0) {
+          v = ca->state[tid];
+        } else {
+          v = ca->noise[(c - 1) * A + tid];
+          p.x[c * A + tid] = v;
+        }
+        xs[tid] = v;
+      }
+      named_sync();
+      pi0_row_in(p, c, 0, xs, tid);
+    } else if (c < M) {
       if (tid < A) {
         const float v = ca->noise[c * A + tid];
         p.x[c * A + tid] = v;
@@ -741,6 +835,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int n = tid; n < D; n += NCOMP) p.h[(size_t)c * D + n] = 0.f;
     }
     grid_sync(p, p.bar, ctl, epoch, ncta, tid);
+    if (p.pi0) {
+      pi0_ato(p, sm, c, M, tid);
+      grid_sync(p, p.bar, ctl, epoch, ncta, tid);
+    }
 
     for (int k = 0; k < S; ++k) {
       for (int l = 0; l < L; ++l) {
@@ -827,7 +925,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // ---- final AdaRMS + action_out_proj (dt folded) + Euler; next step's action_in.
       // CTA c < M owns token row c; thread t owns elements 4t..4t+3 of it.
-      if (c < M) {
+      if (p.pi0 && c == 0) {
+        // π0 state row: no action of its own; the next step restarts it from the state
+        if (p.trace != nullptr && k == p.trace_step) {
+          const int n0 = tid * 4;
+          *reinterpret_cast<float4 *>(p.trace + (size_t)L * C * D + n0) =
+              __ldcg(reinterpret_cast<const float4 *>(p.h + n0));
+        }
+        if (k < S - 1) {
+          float *xr = reinterpret_cast<float *>(sm.op);
+          if (tid < A) xr[tid] = ca->state[tid];
+          named_sync();
+          pi0_row_in(p, 0, k + 1, xr, tid);
+        }
+      } else if (c < M) {
         float *red = reinterpret_cast<float *>(sm.op);  // [8 warps][33]
         float *xr = red + 8 * 33;
         const int n0 = tid * 4;
@@ -875,10 +986,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float nx = __ldcg(p.x + c * A + tid) + v + __ldg(p.b_out + tid);
           p.x[c * A + tid] = nx;
           xr[tid] = nx;
-          if (k == S - 1 && ca->actions != nullptr) ca->actions[c * A + tid] = nx;
+          if (k == S - 1 && ca->actions != nullptr) ca->actions[(c - p.pi0) * A + tid] = nx;
         }
         named_sync();
-        if (k < S - 1) {
+        if (k < S - 1 && p.pi0) {
+          pi0_row_in(p, c, k + 1, xr, tid);
+        } else if (k < S - 1) {
           uint4 wi[4][4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
@@ -902,6 +1015,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (k < S - 1) grid_sync(p, p.bar, ctl, epoch, ncta, tid);
+      if (k < S - 1 && p.pi0) {
+        pi0_ato(p, sm, c, M, tid);
+        grid_sync(p, p.bar, ctl, epoch, ncta, tid);
+      }
     }
   }
   tc_fence_before();

@@ -37,6 +37,12 @@ struct PersistParams {
   // every layer to trace, f32 [L + 1][C][1024]; null in normal calls
   float *trace;
   int trace_step;
+  // π0 suffix (pi0 = 1): row 0 is the state token, rows 1 .. C-1 the action tokens; each
+  // step's action tokens are W_ato SiLU(W_fold x + c_k) + b_ato, the state token W_st s + b_st
+  int pi0;
+  const float *w_fold, *c_tab, *b_ato, *b_st;  // fp32 [1024][32], [S][1024], [1024], [1024]
+  const bf16 *w_ato, *w_st;                    // bf16 [1024][1024], [1024][32]
+  bf16 *op_ato;                                // bf16 [64][1024]: SiLU(W_fold x + c_k) per row
 };
 
 int persistent_smem_bytes();

@@ -457,6 +457,16 @@ cudaError_t launch_persistent(rtvla_ctx *c, CallArgs *dargs, const rtvla_kv *kv,
   p.max_phases = c->pk_max_phases;
   p.trace = trace;
   p.trace_step = trace_step;
+  if (c->variant == RTVLA_VARIANT_PI0) {
+    p.pi0 = 1;
+    p.w_fold = c->pi_wfold;
+    p.c_tab = c->pi_ctab;
+    p.b_ato = c->pi_bato;
+    p.b_st = c->pi_bst;
+    p.w_ato = c->pi_wato;
+    p.w_st = c->pi_wst;
+    p.op_ato = c->op;
+  }
   return persistent_launch(c->pmaps, p, c->sm_count, st);
 }
 
@@ -841,7 +851,7 @@ rtvla_status create_impl(rtvla_ctx *c, const rtvla_weights *w) {
 
   // ---- persistent engine (batch 1, chunk <= 64): norm statistics and attention partials
   if (persistent_init_attributes() != cudaSuccess) return RTVLA_ERR_CUDA;
-  c->pers_ok = c->variant == RTVLA_VARIANT_PI05 && C <= 64 && persistent_fits(c->sm_count);
+  c->pers_ok = C <= 64 && persistent_fits(c->sm_count);
   if (c->pers_ok) {
     const int sp = persistent_max_splits(c->sm_count);
     c->ss_attn = dalloc<float>(c, 64);
@@ -1040,6 +1050,7 @@ rtvla_status rtvla_sample_actions_host(rtvla_ctx *c, const float *noise, const v
                                        const int32_t *valid_len, int batch, int prefix_cap, float *actions_out,
                                        void *stream) {
   if (!c || !noise || !kv_k || !kv_v || !valid_len || !actions_out) return RTVLA_ERR_INVALID_ARG;
+  if (c->variant != RTVLA_VARIANT_PI05) return RTVLA_ERR_INVALID_ARG;  // π0 needs the state
   if (batch < 1 || prefix_cap < 1) return RTVLA_ERR_INVALID_ARG;
   if (batch > c->Bmax || prefix_cap > c->Pmax) return RTVLA_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1270,6 +1281,7 @@ extern "C" rtvla_status rtvla_sample_actions_host_static(rtvla_ctx *c, const flo
                                                          const void *kv_v, const int32_t *valid_len, int batch,
                                                          int prefix_cap, float *actions_out, void *stream) {
   if (!c || !noise || !kv_k || !kv_v || !valid_len || !actions_out) return RTVLA_ERR_INVALID_ARG;
+  if (c->variant != RTVLA_VARIANT_PI05) return RTVLA_ERR_INVALID_ARG;  // π0 needs the state
   if (batch < 1 || prefix_cap < 1) return RTVLA_ERR_INVALID_ARG;
   if (batch > c->Bmax || prefix_cap > c->Pmax) return RTVLA_ERR_SHAPE;
   if (c->engine == RTVLA_ENGINE_PERSISTENT && !use_persistent(c, batch)) return RTVLA_ERR_UNSUPPORTED;

@@ -70,7 +70,7 @@ enum {
   RTVLA_VARIANT_PI05 = 0, /* AdaRMS (scale, shift, gate) from the time MLP; gated residuals */
   RTVLA_VARIANT_PI0 = 1   /* suffix = [state token ; actions]; action tokens from the action-time
                              MLP; plain RMSNorm (scale 1 + w); ungated residuals; final norm.
-                             Runs on the layered engine (AUTO picks it; PERSISTENT is refused) */
+                             Both engines; the persistent one needs chunk + 1 <= 64 */
 };
 
 /*
@@ -213,8 +213,9 @@ rtvla_status rtvla_sample_actions(rtvla_ctx *ctx, const float *noise, const rtvl
  * suffix token, at positions Lv + i with the state at i = 0), then a final RMSNorm and
  * action_out_proj on the action tokens, and x += dt * v.  noise, actions_out: device f32
  * [batch][chunk][action_dim]; state: device f32 [batch][action_dim].  Errors: INVALID_ARG,
- * SHAPE, UNSUPPORTED (a π0.5 context, or engine PERSISTENT); device-detected errors through
- * rtvla_sync_status.  rtvla_sample_actions on a π0 context returns INVALID_ARG (no state).
+ * SHAPE, UNSUPPORTED (a π0.5 context, or engine PERSISTENT with chunk + 1 > 64 or batch > 1);
+ * device-detected errors through rtvla_sync_status.  rtvla_sample_actions on a π0 context returns
+ * INVALID_ARG (no state).
  */
 rtvla_status rtvla_sample_actions_pi0(rtvla_ctx *ctx, const float *noise, const float *state,
                                       const rtvla_kv *kv, float *actions_out, void *stream);
@@ -224,7 +225,8 @@ rtvla_status rtvla_sample_actions_pi0(rtvla_ctx *ctx, const float *noise, const 
  * cache (host bf16 k and v [n_layers][batch][prefix_cap][head_dim], host int32 valid_len
  * [batch]) to the context's device staging, runs the loop, copies the actions back to
  * actions_out (host f32) and waits for the stream.  Host buffers should be pinned for full
- * copy speed.  The staging cache is allocated on first use (RTVLA_ERR_OOM on failure).
+ * copy speed.  The staging cache is allocated on first use (RTVLA_ERR_OOM on failure).  A π0
+ * context returns RTVLA_ERR_INVALID_ARG (this call carries no state).
  */
 rtvla_status rtvla_sample_actions_host(rtvla_ctx *ctx, const float *noise, const void *kv_k,
                                        const void *kv_v, const int32_t *valid_len, int batch,
@@ -248,7 +250,8 @@ rtvla_status rtvla_sample_actions_host(rtvla_ctx *ctx, const float *noise, const
  * per kernel).
  *
  * Arguments, layout and result are those of rtvla_sample_actions_host (host buffers, the
- * call waits for `stream`).  The device of `ctx` must be current.  Errors: INVALID_ARG;
+ * call waits for `stream`).  The device of `ctx` must be current.  Errors: INVALID_ARG (also for
+ * a π0 context: this call carries no state);
  * SHAPE when batch or prefix_cap exceed the context's capacity or when noise + actions +
  * valid_len + K + V (each rounded up to 256 bytes) need more than 32 MiB, checked before
  * anything is copied; UNSUPPORTED when the engine is PERSISTENT and the call is one it
