@@ -8,7 +8,9 @@
 // KV head), one contiguous split of the keys.  K/V chunks of 64 keys are staged in shared
 // memory once and read by all 8 warps; S = Q K^T and O = P V run on mma.sync tensor-core
 // tiles with an online (flash) softmax in fp32.  Several splits are merged by a second
-// kernel with log-sum-exp weights.
+// kernel with log-sum-exp weights.  Calls with at least 64 (sample, query block) units run the
+// tcgen05 kernel of attention_tc.cu instead (attn_launch decides); both write the same
+// partials, so k_attn_combine serves either.
 #include "common.cuh"
 #include "kernels.h"
 

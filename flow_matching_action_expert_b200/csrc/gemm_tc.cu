@@ -10,9 +10,12 @@
 // "res + (x @ W) * gate" of the Realtime-VLA tech blog, kernel list "matmul_small_res_gate").
 //
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer and TMEM owner, warps 2..5 =
-// epilogue: TMEM -> registers (x gate) -> a [TN tokens][128 features] fp32 tile in the freed
-// pipeline stages -> one TMA bulk reduce-add (split K or accumulate) or bulk store per 64
-// tokens.  Every wait is bounded (DevCtl::timeout_ns).
+// epilogue: TMEM -> registers (x gate) -> a [64 tokens][128 features] fp32 box in shared
+// memory -> one TMA bulk reduce-add (split K or accumulate) or bulk store per 64 tokens.
+// Gated-GELU form (GemmParams::glu, the tech blog's "Gated Linear Layer融合 (§4.2)"): a tile's
+// 128 weight rows are 64 gate rows and the 64 matching up rows, and the epilogue turns the
+// box into bf16 GELU_tanh(r*g + b_g) * (r*u + b_u) for 64 features, stored by one TMA copy.
+// Every wait is bounded (DevCtl::timeout_ns).
 #include "common.cuh"
 #include "kernels.h"
 
