@@ -115,18 +115,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// non-blocking test of the phase of `parity` (never suspends the thread)
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 // Waits for the phase of `parity` to complete; gives up after ctl->timeout_ns, records a
 // timeout in the error word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, DevCtl *ctl, int where) {
@@ -158,11 +146,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
-__device__ __forceinline__ uint64_t policy_evict_normal() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
 // 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16)
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -176,13 +159,6 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
 // L2 prefetch of a contiguous range (16-byte aligned, size a multiple of 16): no completion.
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-// L2 prefetch of one 2-D tensor-map box: no shared memory, no barrier, no completion.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *m, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y)
-               : "memory");
 }
 // 2-D tiled load of box (x = inner coordinate in elements, y = row) into shared memory;
 // completes transaction bytes on `bar`.  x * sizeof(elem) must be a multiple of 16.
@@ -217,13 +193,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
                "r"(smem_u32(src)), "r"(x), "r"(y)
-               : "memory");
-}
-// 1-D bulk copy shared -> global (16-byte aligned addresses, size a multiple of 16), in the
-// current bulk async-group
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
-               "r"(bytes)
                : "memory");
 }
 // wait until at most N committed bulk groups are still reading their shared-memory source
