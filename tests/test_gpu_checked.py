@@ -3,8 +3,9 @@
 Checked mode (RTVLA_CHECKED=1 at rtvla_create) places every library buffer between guard
 bands and verifies them in rtvla_sync_status; it stands in for an out-of-bounds / race
 detector.  The bands must survive every engine (persistent kernel, layered graph at batch 1
-and at a ragged batch, the batch-16 kernels: tcgen05 attention and the gated-GELU GEMM) and
-the prefix pass, and a planted overwrite past the residual-stream buffer must be reported
+and at a ragged batch, the batch-16 kernels: tcgen05 attention and the gated-GELU GEMM, π0 on
+both engines) and the prefix pass, and a planted overwrite past the residual-stream buffer
+must be reported
 as RTVLA_ERR_GUARD_OVERWRITE, after which the context still works.
 
 RTVLA_DEVICE_MEMORY_CAP caps the context's device memory: rtvla_create must then return
@@ -74,6 +75,23 @@ def test_guard_bands_hold_on_the_batched_layered_kernels(monkeypatch):
     assert R.rtvla_sync_status(m.ctx) == 0
     assert_actions_close(out, O.sample_actions(WL.as_f32(bits), wl.expert, noise, kf, vf, vnp), wl.name)
     m.close()
+
+
+def test_guard_bands_hold_on_the_pi0_engines(monkeypatch):
+    # π0 (state token + action-time output linear) on the persistent kernel and the layered graph
+    monkeypatch.setenv("RTVLA_CHECKED", "1")
+    wl = WL.workload(1)
+    bits = WL.pi0_expert_weights(wl.expert, bias_std=0.02)
+    wf = WL.as_f32(bits)
+    k, v, valid, kf, vf, vnp = device_kv(wl, pad_fill=3.0e4)
+    noise, state = WL.noise(wl), WL.state(wl)
+    ref = O.pi0_sample_actions(wf, wl.expert, noise, state, kf, vf, vnp)
+    for eng in (R.ENGINE_PERSISTENT, R.ENGINE_LAYERED):
+        m = GpuModel(wl, bits, engine=eng, variant=R.VARIANT_PI0)
+        out = m.sample_pi0(noise, state, k, v, valid)
+        assert R.rtvla_sync_status(m.ctx) == 0
+        assert_actions_close(out, ref, f"checked π0 engine {eng}")
+        m.close()
 
 
 def test_plant_hook_needs_checked_mode(monkeypatch):
