@@ -5,8 +5,7 @@ bands and verifies them in rtvla_sync_status; it stands in for an out-of-bounds 
 detector.  The bands must survive every engine (persistent kernel, layered graph at batch 1
 and at a ragged batch, the batch-16 kernels: tcgen05 attention and the gated-GELU GEMM, π0 on
 both engines) and the prefix pass, and a planted overwrite past the residual-stream buffer
-must be reported
-as RTVLA_ERR_GUARD_OVERWRITE, after which the context still works.
+must be reported as RTVLA_ERR_GUARD_OVERWRITE, after which the context still works.
 
 RTVLA_DEVICE_MEMORY_CAP caps the context's device memory: rtvla_create must then return
 RTVLA_ERR_OOM and free everything it had allocated.
