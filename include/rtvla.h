@@ -173,6 +173,10 @@ typedef struct {
  * concatenated, dt folded into action_out_proj, RoPE cos/sin — and allocates every
  * activation buffer once [BLOG "Static buffers"].  Synchronous.  On success *out owns
  * device memory until rtvla_destroy.  Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA.
+ * Environment read here: RTVLA_WAIT_TIMEOUT_US (bound on every device wait, default
+ * 2,000,000), RTVLA_CHECKED and RTVLA_DEVICE_MEMORY_CAP (see rtvla_sync_status),
+ * RTVLA_PHASE_STAMPS=<file> (persistent-kernel phase timestamps, written by rtvla_destroy),
+ * RTVLA_PAIR_GEMM=1 (the SM-pair form of the layered GEMM; off by default, measured slower).
  */
 rtvla_status rtvla_create(const rtvla_weights *w, const rtvla_config *cfg, rtvla_ctx **out);
 
