@@ -14,6 +14,9 @@ Recipe (all seeds derive from synth.gen.BASE_SEED and the tensor's name):
   * valid prefix lengths: per workload below (3-view: 768 + u_b, u_b uniform in {0..48}).
   * noise: float32 N(0, 1), [B][C][32].
   * prefill embeddings: bf16 N(0, 1) * sqrt(2048), [B][P][2048]; pad mask 1 on valid tokens.
+  * image front-end (SigLIP-shaped tower, ``VisionShape``): float32 pixels uniform in [-1, 1),
+    [N][3][224][224]; weights as ``vision_weights`` states (matrices and biases N(0, 0.02^2),
+    LayerNorm gains near 1).
 """
 from __future__ import annotations
 
@@ -232,7 +235,97 @@ def as_f32(bits_dict: dict) -> dict:
     return {k: gen.bf16_to_f32(v) for k, v in bits_dict.items()}
 
 
+# ----------------------------------------------------------------------------------------
+# image front-end: SigLIP vision tower + multi_modal_projector
+
+@dataclass(frozen=True)
+class VisionShape:
+    """SigLIP-So400m/14-shaped tower.  The pages give 400M parameters, 27 layers, width 1152,
+    224 x 224 images -> 256 tokens and the 1152 -> 2048 projector; patch 14, 16 heads x 72 and
+    MLP 4304 are the public So400m/14 values (they give 412M parameters)."""
+    n_layers: int = 27
+    width: int = 1152
+    mlp_dim: int = 4304
+    n_heads: int = 16
+    patch: int = 14
+    image: int = 224
+    channels: int = 3
+    out_width: int = 2048
+    ln_eps: float = 1e-6
+
+    @property
+    def head_dim(self) -> int:
+        return self.width // self.n_heads
+
+    @property
+    def tokens(self) -> int:
+        return (self.image // self.patch) ** 2
+
+
+def vision_weight_shapes(s: VisionShape) -> dict:
+    W, Fv, p, c = s.width, s.mlp_dim, s.patch, s.channels
+    shapes = {"vis.patch_w": (W, c, p, p), "vis.patch_b": (W,), "vis.pos": (s.tokens, W),
+              "vis.post_w": (W,), "vis.post_b": (W,),
+              "vis.proj_w": (s.out_width, W), "vis.proj_b": (s.out_width,)}
+    for l in range(s.n_layers):
+        shapes.update({
+            f"vis{l}.ln1_w": (W,), f"vis{l}.ln1_b": (W,),
+            f"vis{l}.wq": (W, W), f"vis{l}.bq": (W,), f"vis{l}.wk": (W, W), f"vis{l}.bk": (W,),
+            f"vis{l}.wv": (W, W), f"vis{l}.bv": (W,), f"vis{l}.wo": (W, W), f"vis{l}.bo": (W,),
+            f"vis{l}.ln2_w": (W,), f"vis{l}.ln2_b": (W,),
+            f"vis{l}.fc1_w": (Fv, W), f"vis{l}.fc1_b": (Fv,), f"vis{l}.fc2_w": (W, Fv), f"vis{l}.fc2_b": (W,),
+        })
+    return shapes
+
+
+def _vision_kind(name: str) -> str:
+    leaf = name.split(".", 1)[1]
+    if leaf in ("ln1_w", "ln2_w", "post_w"):
+        return "ln_gain"
+    if leaf in ("ln1_b", "ln2_b", "post_b"):
+        return "ln_bias"
+    if leaf == "pos":
+        return "pos"
+    if leaf in ("patch_b", "bq", "bk", "bv", "bo", "fc1_b", "fc2_b", "proj_b"):
+        return "bias"
+    return "matrix"
+
+
+def vision_weights(s: VisionShape, std: float = 0.02, stressed: bool = False, tag: str = "vision") -> dict:
+    """bf16 bit patterns of every vision tensor.
+
+    Matrices N(0, std^2) ("stressed": W_q and W_k at 3 std, so attention is peaked rather
+    than near-uniform); biases N(0, std^2); position embedding N(0, 0.1^2); LayerNorm
+    gains 1 + N(0, 0.1^2) and offsets N(0, 0.05^2), so every affine term is exercised.
+    """
+    out = {}
+    for name, shape in vision_weight_shapes(s).items():
+        kind = _vision_kind(name)
+        key = f"{tag}/{name}"
+        if kind == "ln_gain":
+            out[name] = gen.bf16_bits(1.0 + gen.normal(key, shape, 0.1))
+        elif kind == "ln_bias":
+            out[name] = gen.normal_bf16(key, shape, 0.05)
+        elif kind == "pos":
+            out[name] = gen.normal_bf16(key, shape, 0.1)
+        elif kind == "bias":
+            out[name] = gen.normal_bf16(key, shape, std)
+        else:
+            scale = 3.0 if stressed and name.split(".", 1)[1] in ("wq", "wk") else 1.0
+            out[name] = gen.normal_bf16(key, shape, std * scale)
+    return out
+
+
+def images(s: VisionShape, n: int, tag: str = "images") -> np.ndarray:
+    """float32 pixels uniform in [-1, 1), [n][channels][image][image]: the camera frames after
+    the resize and the [-1, 1] normalisation, which are not part of the path."""
+    shape = (n, s.channels, s.image, s.image)
+    u = gen.uniform(f"{tag}/{n}", int(np.prod(shape)))
+    return (2.0 * u - 1.0).astype(np.float32).reshape(shape)
+
+
 __all__ = ["ExpertShape", "PrefillShape", "Workload", "workload", "expert_weights",
            "pi0_expert_weight_shapes", "pi0_expert_weights", "state",
            "prefill_weights", "kv_cache", "noise", "prefill_inputs", "as_f32",
-           "expert_weight_shapes", "prefill_weight_shapes", "replace", "field"]
+           "expert_weight_shapes", "prefill_weight_shapes", "replace", "field",
+           "VisionShape", "vision_weight_shapes", "vision_weights", "images"]
