@@ -40,11 +40,16 @@ def parse():
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--engine", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--workload", default="2-view", choices=["2-view", "1-view", "3-view", "e2e", "stream", "pi0"],
+    p.add_argument("--workload", default="2-view",
+                   choices=["2-view", "1-view", "3-view", "e2e", "stream", "pi0", "vision", "pipeline"],
                    help="2-view (the headline line), 1-view, 3-view (with --batch), e2e: prefill of the "
                         "544-token prefix, then the denoise loop; stream: frames of e2e back to back, the "
                         "prefill of frame n+1 overlapping the denoise of frame n (layered engine); pi0: the "
-                        "2-view workload on the pi0 suffix variant (state token, action-time MLP)")
+                        "2-view workload on the pi0 suffix variant (state token, action-time MLP); vision: "
+                        "the image encoder (27-layer SigLIP tower + projector) on --views views; pipeline: "
+                        "full pi0 inference on --views views (image encoder, prefix pass over the image "
+                        "tokens with an empty prompt, 10-step pi0 loop, chunk 63)")
+    p.add_argument("--views", type=int, default=2, choices=[1, 2, 3])
     return p.parse_args()
 
 
@@ -91,6 +96,15 @@ def prefill_algorithmic(wl):
     return bytes_, flops
 
 
+def prefill_kernels(n_layers):
+    """Kernels of one rtvla_prefill graph at the sizes benched here (the attention split into
+    several key ranges, the gate/up GEMM with the GELU epilogue): the mask and embedding
+    kernels; per layer RMSNorm, QKV GEMM and QKV post; per full layer (all but the last)
+    attention, its split combine, O GEMM, RMSNorm, gate/up GEMM and down GEMM.  158 at 18
+    layers, as the ncu launch list of the 544-token prefill counts."""
+    return 2 + 3 * n_layers + 6 * (n_layers - 1)
+
+
 def pi0_algorithmic(wl):
     """Bytes and FLOPs of one 10-step pi0 loop: the 18 layers' weights, the folded action-time
     MLP (fp32 W_fold [1024][32] and its output linear), state and action projections, the
@@ -126,6 +140,21 @@ def algorithmic(wl):
     attn_flops = sum(4 * H * wl.chunk * (l + wl.chunk) * hd for l in wl.valid_lens) * L
     flops_step = 2 * M * params + attn_flops
     return bytes_step * S, flops_step * S, w_bytes * S
+
+
+def vision_algorithmic(vcfg, n_img):
+    """Bytes and FLOPs of one encode of n_img images: every weight matrix read once (bf16), the
+    images read (f32) and the embeddings written (bf16); 2 * tokens * MACs of the patch
+    convolution, the 27 layers' linears and the projector, plus 4 * heads * 256^2 * 72 of
+    attention per image and layer."""
+    W, Fv, L, T = vcfg.width, vcfg.mlp_dim, vcfg.n_layers, vcfg.tokens
+    patch = W * vcfg.channels * vcfg.patch ** 2
+    layer = 4 * W * W + 2 * W * Fv
+    proj = vcfg.out_width * W
+    tok = n_img * T
+    flops = 2 * tok * (patch + L * layer + proj) + L * n_img * 4 * vcfg.n_heads * T * T * vcfg.head_dim
+    bytes_ = (patch + L * layer + proj) * 2 + n_img * vcfg.channels * vcfg.image ** 2 * 4 + tok * vcfg.out_width * 2
+    return bytes_, flops
 
 
 def reduce_max(vals, device):
@@ -291,6 +320,11 @@ class OracleLoop:
 def run_reference(args, rank):
     if rank != 0:
         return
+    if args.workload in ("vision", "pipeline"):
+        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the denoise workloads; the "
+                          "image encoder's fp64 oracle is timed as the cpu_baseline of the repo arm's vision line"}),
+              flush=True)
+        return
     wl = workload(args.batch, args.workload if args.workload not in ("e2e", "stream") else "2-view")
     loop = OracleLoop(wl)
     for _ in range(args.warmup):
@@ -320,6 +354,10 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.workload == "vision":
+        return run_vision(args, rank, world, local_rank)
+    if args.workload == "pipeline":
+        return run_pipeline(args, rank, world, local_rank)
     wl = workload(args.batch, args.workload)
     if args.workload == "e2e":
         return run_e2e(args, rank, world, local_rank, wl)
@@ -612,7 +650,7 @@ def run_e2e(args, rank, world, local_rank, wl):
     st = R.rtvla_sync_status(ctx, stream)
     if st != 0:
         raise RuntimeError(f"device status {R.STATUS[st]}")
-    kernels = R.rtvla_kernels_per_call(ctx, wl.batch)
+    kernels = R.rtvla_kernels_per_call(ctx, wl.batch) + prefill_kernels(wl.prefill.n_layers)
     R.rtvla_destroy(ctx)
     if rank != 0:
         return
@@ -637,6 +675,7 @@ def run_e2e(args, rank, world, local_rank, wl):
                      "algorithmic_bytes_per_launch": int(pb), "roofline_ms": round(t_pre * 1e3, 4),
                      "denoise_roofline_ms": round(t_den * 1e3, 4),
                      "denoise_frac": round(t_den * 1e3 / den_ms, 4)},
+        "gpu_launches": kernels * args.steps,
         "kernels_per_step": kernels,
         "clocks": clk.summary(),
     }
@@ -728,6 +767,263 @@ def run_stream(args, rank, world, local_rank, wl):
         "config": workload_config(wl, world), "engine": "layered (prefill and denoise graphs on two streams)",
         "sequential_ms_per_frame": round(seq_ms, 4), "pipelined_ms_per_frame": round(pip_ms, 4),
         "overlap_gain": round(seq_ms / pip_ms, 3), "pipelined_vs_sequential_max_abs": diff,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _vision_ctx(vcfg, n_img, dev, tag="vision"):
+    import torch
+
+    import flow_matching_action_expert_b200 as R
+    from synth import workloads as WL
+    bits = WL.vision_weights(vcfg, tag=tag)
+    dw = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev) for k, v in bits.items()}
+    ctx = R.rtvla_vision_create(dw, R.make_vision_config(n_layers=vcfg.n_layers, max_images=n_img))
+    del dw
+    return ctx, bits
+
+
+def run_vision(args, rank, world, local_rank):
+    """The image encoder alone: --views camera views (one sample) through the 27-layer SigLIP
+    tower and the projector into a prefix buffer, one rtvla_encode_images call (one graph
+    replay) per step, inputs resident.  e2e: the images copied from pinned host memory and the
+    embeddings read back, every step."""
+    import torch
+
+    import flow_matching_action_expert_b200 as R
+    from synth import workloads as WL
+
+    dev = torch.device("cuda", local_rank)
+    vcfg = WL.VisionShape()
+    V = args.views
+    ctx, bits = _vision_ctx(vcfg, V, dev)
+    imgs_np = WL.images(vcfg, V)
+    imgs = torch.from_numpy(imgs_np).to(dev)
+    P = V * vcfg.tokens
+    emb = torch.zeros((1, P, vcfg.out_width), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def call():
+        R.rtvla_encode_images(ctx, imgs, 1, V, emb, P, stream)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    st = R.rtvla_vision_sync_status(ctx, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {R.STATUS[st]}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    times = [a.elapsed_time(b) for a, b in ev]
+    # end to end: pinned host images in, embeddings out, every step
+    h_imgs = torch.from_numpy(imgs_np).pin_memory()
+    h_emb = torch.empty(emb.shape, dtype=emb.dtype).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e2e_ev[i][0].record(stream)
+        imgs.copy_(h_imgs, non_blocking=True)
+        call()
+        h_emb.copy_(emb, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_times = [a.elapsed_time(b) for a, b in e2e_ev]
+    ms, e2e_ms = reduce_max([statistics.mean(times), statistics.mean(e2e_times)], dev)
+    st = R.rtvla_vision_sync_status(ctx, stream)
+    if st != 0:
+        raise RuntimeError(f"device status {R.STATUS[st]}")
+    kernels = R.rtvla_vision_kernels_per_call(ctx, V)
+    R.rtvla_vision_destroy(ctx)
+    if rank != 0:
+        return
+    hbm, bf16_pk, bf16_sus, src = peaks()
+    vb, vf = vision_algorithmic(vcfg, V)
+    t_roof = max(vb / (hbm * 1e9), vf / (bf16_pk * 1e12))
+    achieved = vf / (ms * 1e-3) / 1e12
+    line = {
+        "metric": f"image encoder latency ms ({V}-view, 27-layer SigLIP tower + projector)",
+        "value": round(ms, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform [-1,1) f32 pixels)",
+        "config": {"workload": f"SigLIP-So400m/14 shape, {V} x 224x224 views -> {P} prefix embeddings",
+                   "layers": vcfg.n_layers, "width": vcfg.width, "mlp": vcfg.mlp_dim, "heads": vcfg.n_heads,
+                   "images": V, "tokens": P, "parallelism": f"replicas{world}"},
+        "l2": "flushed by a 256 MiB write between timed steps",
+        "roofline": {"bound": "tensor", "kernel": "rtvla_encode_images (tcgen05 GEMMs + attention, one graph)",
+                     "achieved": round(achieved, 1), "peak": bf16_pk, "unit": "TFLOP/s",
+                     "frac": round(achieved / bf16_pk, 4), "traffic": None, "peak_source": src,
+                     "algorithmic_flops_per_launch": int(vf), "algorithmic_bytes_per_launch": int(vb),
+                     "roofline_ms": round(t_roof * 1e3, 4)},
+        "e2e": {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": int(imgs.numel() * 4),
+                "d2h_bytes_per_step": int(emb.numel() * 2)},
+        "gpu_launches": kernels * args.steps,
+        "kernels_per_step": kernels,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        from oracle import vision as OV
+        W = WL.as_f32(bits)
+        t0 = time.perf_counter()
+        OV.encode_image(imgs_np[0], W, vcfg)
+        one = (time.perf_counter() - t0) * 1e3
+        line["cpu_baseline"] = {"value": round(one * V, 1), "unit": "ms", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"1 of the {V} images through the fp64 oracle tower, scaled by {V}"}
+    print(json.dumps(line), flush=True)
+
+
+PAGES_PI0_MS = {1: 20.0, 2: 27.3, 3: 36.8}   # Realtime-VLA, full π0 inference on one RTX 4090
+
+
+def run_pipeline(args, rank, world, local_rank):
+    """Full π0 inference as the pages time it (empty prompt, chunk 63, 10 steps, batch 1):
+    --views camera views -> image encoder -> prefix pass over the views * 256 image tokens
+    (Gemma-2B shape, 18 layers) -> the π0 10-step loop (the persistent kernel).  value: device
+    time per inference with inputs resident; e2e: the same with images, robot state and noise
+    copied from pinned host memory and the actions copied back, every step."""
+    import torch
+
+    import flow_matching_action_expert_b200 as R
+    from synth import workloads as WL
+
+    dev = torch.device("cuda", local_rank)
+    V = args.views
+    vcfg = WL.VisionShape()
+    P = V * vcfg.tokens
+    wl = WL.Workload(f"pi0 pipeline {V}-view: SigLIP L27 + prefill P{P} + L18 C63 B1", WL.ExpertShape(), 63, 1, P,
+                     (P,), prefill=WL.PrefillShape(), description="empty prompt")
+    vctx, _ = _vision_ctx(vcfg, V, dev)
+    bits = WL.pi0_expert_weights(wl.expert, bias_std=0.02)
+    bits.update(WL.prefill_weights(wl.prefill))
+    dw = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev) for k, v in bits.items()}
+    del bits
+    cfg = R.make_config(n_layers=wl.expert.n_layers, chunk=wl.chunk, max_prefix=P, max_batch=1, has_prefill=True,
+                        engine=args.engine, variant=R.VARIANT_PI0)
+    ctx = R.rtvla_create(dw, cfg)
+    del dw
+    torch.cuda.empty_cache()
+    imgs_np, noise_np, state_np = WL.images(vcfg, V), WL.noise(wl), WL.state(wl)
+    imgs = torch.from_numpy(imgs_np).to(dev)
+    noise = torch.from_numpy(noise_np).to(dev)
+    state = torch.from_numpy(state_np).to(dev)
+    out = torch.empty_like(noise)
+    emb = torch.zeros((1, P, 2048), dtype=torch.bfloat16, device=dev)
+    mask = torch.ones((1, P), dtype=torch.uint8, device=dev)
+    L = wl.expert.n_layers
+    k = torch.zeros((L, 1, P, 256), dtype=torch.bfloat16, device=dev)
+    v = torch.zeros_like(k)
+    valid = torch.zeros(1, dtype=torch.int32, device=dev)
+    kv = R.make_kv(k, v, valid, 1, P)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        R.rtvla_encode_images(vctx, imgs, 1, V, emb, P, stream)
+        if ev:
+            ev[1].record(stream)
+        R.rtvla_prefill(ctx, emb, mask, 1, P, kv, stream)
+        if ev:
+            ev[2].record(stream)
+        R.rtvla_sample_actions_pi0(ctx, noise, state, kv, out, stream)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    for c, f in ((vctx, R.rtvla_vision_sync_status), (ctx, R.rtvla_sync_status)):
+        st = f(c, stream)
+        if st != 0:
+            raise RuntimeError(f"device status {R.STATUS[st]}")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            step(evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    vis = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    pre = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    den = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    tot = statistics.mean(e[0].elapsed_time(e[3]) for e in evs)
+    # end to end: pinned host images, state and noise in, actions out, every step
+    h_imgs = torch.from_numpy(imgs_np).pin_memory()
+    h_state = torch.from_numpy(state_np).pin_memory()
+    h_noise = torch.from_numpy(noise_np).pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e2e_ev[i][0].record(stream)
+        imgs.copy_(h_imgs, non_blocking=True)
+        state.copy_(h_state, non_blocking=True)
+        noise.copy_(h_noise, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e = statistics.mean(a.elapsed_time(b) for a, b in e2e_ev)
+    tot, vis, pre, den, e2e = reduce_max([tot, vis, pre, den, e2e], dev)
+    for c, f in ((vctx, R.rtvla_vision_sync_status), (ctx, R.rtvla_sync_status)):
+        st = f(c, stream)
+        if st != 0:
+            raise RuntimeError(f"device status {R.STATUS[st]}")
+    kernels = (R.rtvla_vision_kernels_per_call(vctx, V) + prefill_kernels(wl.prefill.n_layers)
+               + R.rtvla_kernels_per_call(ctx, 1))
+    R.rtvla_vision_destroy(vctx)
+    R.rtvla_destroy(ctx)
+    if rank != 0:
+        return
+    hbm, bf16_pk, bf16_sus, src = peaks()
+    vb, vf = vision_algorithmic(vcfg, V)
+    pb, pf = prefill_algorithmic(wl)
+    db, df = pi0_algorithmic(wl)
+    t_vis = max(vb / (hbm * 1e9), vf / (bf16_sus * 1e12)) * 1e3
+    t_pre = max(pb / (hbm * 1e9), pf / (bf16_sus * 1e12)) * 1e3
+    t_den = max(db / (hbm * 1e9), df / (bf16_sus * 1e12)) * 1e3
+    h2d = int(imgs.numel() * 4 + state.numel() * 4 + noise.numel() * 4)
+    line = {
+        "metric": f"full pi0 inference latency ms ({V}-view, empty prompt, chunk 63: image encoder + prefix pass "
+                  f"+ 10-step loop)",
+        "value": round(tot, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(tot, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": round(tot / PAGES_PI0_MS[V], 4),
+        "baseline_context": f"{PAGES_PI0_MS[V]} ms: Realtime-VLA, full pi0 inference on one RTX 4090 (the pages' "
+                            f"Table 1); another machine's number",
+        "dtype": "bf16",
+        "data": "synthetic (seeded bf16 weights, uniform [-1,1) pixels, N(0,1) state and noise)",
+        "config": workload_config(wl, world) | {"views": V, "vision_layers": vcfg.n_layers},
+        "l2": "flushed by a 256 MiB write between timed steps; weights (5.9 GB) exceed L2",
+        "vision_ms": round(vis, 4), "prefill_ms": round(pre, 4), "denoise_ms": round(den, 4),
+        "roofline": {"bound": "tensor", "kernel": "rtvla_encode_images (the stage this line adds)",
+                     "achieved": round(vf / (vis * 1e-3) / 1e12, 1), "peak": bf16_sus, "unit": "TFLOP/s",
+                     "frac": round(vf / (vis * 1e-3) / 1e12 / bf16_sus, 4), "traffic": None, "peak_source": src,
+                     "stage_roofline_ms": {"vision": round(t_vis, 4), "prefill": round(t_pre, 4),
+                                           "denoise": round(t_den, 4)},
+                     "pipeline_frac": round((t_vis + t_pre + t_den) / tot, 4)},
+        "e2e": {"value": round(e2e, 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": kernels * args.steps,
+        "kernels_per_step": kernels,
+        "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
 

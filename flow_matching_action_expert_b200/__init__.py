@@ -29,6 +29,8 @@ EXPORTS = (
     "rtvla_sync_status", "rtvla_debug_trace", "rtvla_kernels_per_call", "rtvla_set_engine",
     "rtvla_set_wait_timeout_us", "rtvla_destroy", "rtvla_status_string", "rtvla_debug_plant_guard_fault",
     "rtvla_sample_actions_pi0", "rtvla_debug_trace_pi0",
+    "rtvla_vision_create", "rtvla_encode_images", "rtvla_vision_debug_trace", "rtvla_vision_sync_status",
+    "rtvla_vision_kernels_per_call", "rtvla_vision_destroy",
 )
 
 
@@ -64,6 +66,22 @@ class RtvlaWeights(ctypes.Structure):
                 + [("final_ln", _P)])
 
 
+class RtvlaVisionConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "n_layers", "width", "mlp_dim", "n_heads", "patch", "image", "out_width", "max_images")] + [
+        ("ln_eps", ctypes.c_float)]
+
+
+_VIS_SINGLE = ("patch_w", "patch_b", "pos")
+_VIS_LAYER = ("ln1_w", "ln1_b", "wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "ln2_w", "ln2_b",
+              "fc1_w", "fc1_b", "fc2_w", "fc2_b")
+_VIS_FINAL = ("post_w", "post_b", "proj_w", "proj_b")
+
+
+class RtvlaVisionWeights(ctypes.Structure):
+    _fields_ = [(n, _P) for n in _VIS_SINGLE] + [(n, _PP) for n in _VIS_LAYER] + [(n, _P) for n in _VIS_FINAL]
+
+
 class RtvlaKV(ctypes.Structure):
     _fields_ = [("k", _P), ("v", _P), ("valid_len", _P), ("batch", ctypes.c_int), ("prefix_cap", ctypes.c_int)]
 
@@ -95,12 +113,22 @@ def _lib():
         lib.rtvla_debug_plant_guard_fault.argtypes = [_P]
         lib.rtvla_destroy.argtypes = [_P]
         lib.rtvla_destroy.restype = None
+        lib.rtvla_vision_create.argtypes = [ctypes.POINTER(RtvlaVisionWeights), ctypes.POINTER(RtvlaVisionConfig),
+                                            ctypes.POINTER(_P)]
+        lib.rtvla_encode_images.argtypes = [_P, _P, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int, _P]
+        lib.rtvla_vision_debug_trace.argtypes = [_P, _P, ctypes.c_int, _P, _P, _P]
+        lib.rtvla_vision_sync_status.argtypes = [_P, _P]
+        lib.rtvla_vision_kernels_per_call.argtypes = [_P, ctypes.c_int]
+        lib.rtvla_vision_destroy.argtypes = [_P]
+        lib.rtvla_vision_destroy.restype = None
         lib.rtvla_status_string.argtypes = [ctypes.c_int]
         lib.rtvla_status_string.restype = ctypes.c_char_p
         for n in EXPORTS:
-            if n not in ("rtvla_kv_bytes", "rtvla_destroy", "rtvla_status_string", "rtvla_kernels_per_call"):
+            if n not in ("rtvla_kv_bytes", "rtvla_destroy", "rtvla_status_string", "rtvla_kernels_per_call",
+                         "rtvla_vision_destroy", "rtvla_vision_kernels_per_call"):
                 getattr(lib, n).restype = ctypes.c_int
         lib.rtvla_kernels_per_call.restype = ctypes.c_int
+        lib.rtvla_vision_kernels_per_call.restype = ctypes.c_int
         _LIB = lib
     return _LIB
 
@@ -162,6 +190,29 @@ def make_weights(w: dict, n_layers: int):
             arr = (_P * n_layers)(*[_ptr(w[f"pf{l}.{n[3:]}"]) for l in range(n_layers)])
             keep.append(arr)
             setattr(ws, n, ctypes.cast(arr, _PP))
+    return ws, keep
+
+
+def make_vision_config(n_layers=27, max_images=2, ln_eps=1e-6) -> RtvlaVisionConfig:
+    """rtvla_vision_config for the SigLIP-So400m/14 shape (width 1152, MLP 4304, 16 heads, patch 14,
+    224 x 224 images, projector to 2048)."""
+    return RtvlaVisionConfig(n_layers=n_layers, width=1152, mlp_dim=4304, n_heads=16, patch=14, image=224,
+                             out_width=2048, max_images=max_images, ln_eps=ln_eps)
+
+
+def make_vision_weights(w: dict, n_layers: int):
+    """rtvla_vision_weights from a dict of CUDA bf16 tensors named as in synth.workloads
+    ("vis.patch_w", "vis{l}.wq", ...).  Returns (struct, keepalive)."""
+    keep = []
+    ws = RtvlaVisionWeights()
+    for n in _VIS_SINGLE + _VIS_FINAL:
+        setattr(ws, n, _ptr(w.get(f"vis.{n}")))
+    for n in _VIS_LAYER:
+        if not any(f"vis{l}.{n}" in w for l in range(n_layers)):
+            continue
+        arr = (_P * n_layers)(*[_ptr(w.get(f"vis{l}.{n}")) for l in range(n_layers)])
+        keep.append(arr)
+        setattr(ws, n, ctypes.cast(arr, _PP))
     return ws, keep
 
 
@@ -253,3 +304,39 @@ def rtvla_destroy(ctx: int):
 
 def rtvla_status_string(code: int) -> str:
     return _lib().rtvla_status_string(code).decode()
+
+
+# ---------------------------------------------------------------------------------------
+# image front-end
+
+def rtvla_vision_create(weights: dict, cfg: RtvlaVisionConfig) -> int:
+    ws, keep = make_vision_weights(weights, cfg.n_layers)
+    out = _P()
+    _check(_lib().rtvla_vision_create(ctypes.byref(ws), ctypes.byref(cfg), ctypes.byref(out)),
+           "rtvla_vision_create")
+    del keep
+    return out.value
+
+
+def rtvla_encode_images(ctx: int, images, batch: int, views: int, prefix_embeds, prefix_len: int, stream=None):
+    _check(_lib().rtvla_encode_images(ctx, _ptr(images), batch, views, _ptr(prefix_embeds), prefix_len,
+                                      _stream(stream)), "rtvla_encode_images")
+
+
+def rtvla_vision_debug_trace(ctx: int, images, n_images: int, h_layers, prefix_embeds, stream=None):
+    _check(_lib().rtvla_vision_debug_trace(ctx, _ptr(images), n_images, _ptr(h_layers), _ptr(prefix_embeds),
+                                           _stream(stream)), "rtvla_vision_debug_trace")
+
+
+def rtvla_vision_sync_status(ctx: int, stream=None) -> int:
+    """Returns the device status code (0 = ok); does not raise."""
+    return _lib().rtvla_vision_sync_status(ctx, _stream(stream))
+
+
+def rtvla_vision_kernels_per_call(ctx: int, n_images: int) -> int:
+    return _lib().rtvla_vision_kernels_per_call(ctx, n_images)
+
+
+def rtvla_vision_destroy(ctx: int):
+    if ctx:
+        _lib().rtvla_vision_destroy(ctx)

@@ -126,6 +126,32 @@ cudaError_t launch_fold_cols(const bf16 *W, int R, int Kd, const bf16 *gamma, bf
 cudaError_t launch_scale_to_f32(const bf16 *w, int n, double s, float *out, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------
+// image front-end (vision.cu): SigLIP-shaped tower of width 1152, 16 heads x 72, 256 tokens per
+// 224 x 224 image (14 x 14 patches), projector to 2048
+constexpr int VIS_WIDTH = 1152;
+constexpr int VIS_TOKENS = 256;
+constexpr int VIS_PATCH_K = 640;   // the patch operand's 3 x 14 x 14 = 588 values, zero-padded
+constexpr int VIS_MLP_PAD = 4352;  // the MLP width 4304, zero-padded to whole 128-row tiles
+constexpr int VIS_OUT = 2048;
+
+// Per-call pointers of the captured encode graph (written to device memory before each replay).
+struct VisArgs {
+  const float *images;  // [n][3][224][224]
+  bf16 *out;            // prefix embeddings [batch][ld][2048]
+  int views;            // image i -> sample i / views, rows (i % views) * 256 ..
+  int ld;               // prefix rows per sample
+};
+
+cudaError_t vis_init_attributes();
+cudaError_t launch_vis_embed(const VisArgs *va, bf16 *cols, float *h, const float *table, int n_img,
+                             cudaStream_t st);
+cudaError_t launch_vis_ln(float *x, const float *add, const float *gain, const float *offset, bf16 *y, float *acc,
+                          const float *acc_init, int acc_cols, int M, float eps, cudaStream_t st);
+cudaError_t launch_vis_attn(const float *qkv, bf16 *out, int n_img, cudaStream_t st);
+cudaError_t launch_vis_gelu(const float *acc, bf16 *out, int M, int cols, cudaStream_t st);
+cudaError_t launch_vis_out(const VisArgs *va, const float *acc, int n_img, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------
 // checked mode: guard bands of GUARD_BYTES filled with GUARD_FILL before and after every
 // library buffer; the checker flags (DEVERR_GUARD) and refills every band that changed
 constexpr int GUARD_BYTES = 4096;

@@ -326,6 +326,107 @@ void rtvla_destroy(rtvla_ctx *ctx);
 /* Static English text for a status code. */
 const char *rtvla_status_string(rtvla_status s);
 
+/* =========================================================================================
+ * Image front-end: the SigLIP vision tower and the multi_modal_projector, which turn each
+ * camera view into the prefix embeddings rtvla_prefill consumes [BLOG "pi0.5 inference
+ * flow": model structure (SigLIP, 400M parameters, 224 x 224 image -> 256 tokens), encoder
+ * step 1 (256 embeddings per view, scaled by sqrt(2048)) and step 3 (image tokens, then
+ * language tokens); class hierarchy (vision_tower: SiglipVisionTransformer, 27 layers;
+ * multi_modal_projector: Linear 1152 -> 2048)].  A context of its own, independent of
+ * rtvla_ctx; the same conventions (row-major, (out, in) Linear layout, bf16 = IEEE bfloat16,
+ * asynchronous calls on `stream`, device-detected errors through a sync call).
+ *
+ * Per image: h = patch_conv(image) + position embedding (a 14 x 14, stride 14 convolution
+ * 3 -> 1152 with bias; tokens in raster order of the 16 x 16 patch grid); n_layers pre-norm
+ * layers h += o_proj(MHA(LN1(h))), h += fc2(GELU_tanh(fc1(LN2(h)))) with biased q/k/v/o/fc1/
+ * fc2 linears and bidirectional attention over the image's 256 tokens (16 heads x 72, scale
+ * 1/sqrt(72), no mask, no rotary embedding); then embeddings = sqrt(2048) *
+ * (post_LN(h) W_proj^T + b_proj).  LayerNorm: (x - mean) / sqrt(var + ln_eps) * w + b,
+ * biased variance.  The pages name the tower; patch 14, 16 heads and MLP 4304 are the public
+ * SigLIP-So400m/14 shape, which has the pages' 27 layers, width 1152 and ~400M parameters.
+ * ========================================================================================= */
+typedef struct rtvla_vision_ctx rtvla_vision_ctx; /* opaque; owned by the library */
+
+typedef struct {
+  int n_layers;   /* 27 (1..64 accepted) */
+  int width;      /* 1152 */
+  int mlp_dim;    /* 4304 */
+  int n_heads;    /* 16 (head_dim = width / n_heads = 72) */
+  int patch;      /* 14 */
+  int image;      /* 224: (image / patch)^2 = 256 tokens per image, 3 channels */
+  int out_width;  /* 2048: the prefix pass's width */
+  int max_images; /* most images one rtvla_encode_images call encodes (1..64) */
+  float ln_eps;   /* 1e-6 */
+} rtvla_vision_config;
+
+/* Device pointers to bf16 tensors, read only during rtvla_vision_create (the library keeps its
+ * own repacked copies).  Per-layer fields are host arrays of n_layers device pointers. */
+typedef struct {
+  const void *patch_w;          /* [width][3][patch][patch] patch convolution */
+  const void *patch_b;          /* [width] */
+  const void *pos;              /* [256][width] position embedding */
+  const void *const *ln1_w;     /* [L] -> [width]  LayerNorm before attention: gain */
+  const void *const *ln1_b;     /* [L] -> [width]  offset */
+  const void *const *wq;        /* [L] -> [width][width] */
+  const void *const *bq;        /* [L] -> [width] */
+  const void *const *wk;
+  const void *const *bk;
+  const void *const *wv;
+  const void *const *bv;
+  const void *const *wo;        /* [L] -> [width][width] attention output projection */
+  const void *const *bo;
+  const void *const *ln2_w;     /* [L] -> [width]  LayerNorm before the MLP */
+  const void *const *ln2_b;
+  const void *const *fc1_w;     /* [L] -> [mlp_dim][width] */
+  const void *const *fc1_b;     /* [L] -> [mlp_dim] */
+  const void *const *fc2_w;     /* [L] -> [width][mlp_dim] */
+  const void *const *fc2_b;     /* [L] -> [width] */
+  const void *post_w;           /* [width] post_layernorm gain */
+  const void *post_b;           /* [width] */
+  const void *proj_w;           /* [out_width][width] multi_modal_projector */
+  const void *proj_b;           /* [out_width] */
+} rtvla_vision_weights;
+
+/* Creates an image-encoder context: repacks the weights (fc1 / fc2 zero-padded to 4352 MLP
+ * features, the patch operand to 640 values), builds the fp32 table patch bias + position
+ * embedding, and allocates every buffer for max_images images.  Synchronous.  Errors:
+ * INVALID_ARG, UNSUPPORTED (a shape other than the one above), OOM, CUDA.  Reads
+ * RTVLA_WAIT_TIMEOUT_US, RTVLA_CHECKED and RTVLA_DEVICE_MEMORY_CAP as rtvla_create does. */
+rtvla_status rtvla_vision_create(const rtvla_vision_weights *w, const rtvla_vision_config *cfg,
+                                 rtvla_vision_ctx **out);
+
+/*
+ * Encodes batch x views images and writes their embeddings into the prefix buffer of
+ * rtvla_prefill.  images: device f32 [batch][views][3][224][224], pixels after resize and
+ * [-1, 1] normalisation, 4-byte aligned.  prefix_embeds: device bf16
+ * [batch][prefix_len][out_width], 16-byte aligned: view v of sample b fills rows
+ * v * 256 .. v * 256 + 255 of sample b; no other row is written (the caller puts the prompt
+ * embeddings after the image rows).  Runs as one CUDA-graph replay per call (captured on the
+ * first call with this image count).  Errors: INVALID_ARG (null or misaligned pointer, batch
+ * or views < 1), SHAPE (batch * views > max_images, or views * 256 > prefix_len);
+ * device-detected DEVICE_TIMEOUT through rtvla_vision_sync_status.
+ */
+rtvla_status rtvla_encode_images(rtvla_vision_ctx *ctx, const float *images, int batch, int views,
+                                 void *prefix_embeds, int prefix_len, void *stream);
+
+/* Test hook: encodes n_images images of [n][3][224][224] (as one sample of n views) and
+ * writes the residual stream after the embedding and after each layer to h_layers: device f32
+ * [n_layers + 1][n_images * 256][width]; then the embeddings to prefix_embeds as
+ * rtvla_encode_images would (prefix_len = n_images * 256).  Launches the kernels directly
+ * (no graph).  Errors: as rtvla_encode_images. */
+rtvla_status rtvla_vision_debug_trace(rtvla_vision_ctx *ctx, const float *images, int n_images,
+                                      float *h_layers, void *prefix_embeds, void *stream);
+
+/* As rtvla_sync_status, for an image-encoder context (guard bands checked in checked mode). */
+rtvla_status rtvla_vision_sync_status(rtvla_vision_ctx *ctx, void *stream);
+
+/* Kernels of this library one rtvla_encode_images call of n_images images launches (after
+ * such a call has been made once), else -1. */
+int rtvla_vision_kernels_per_call(rtvla_vision_ctx *ctx, int n_images);
+
+/* Frees everything the context owns (waits for the device first).  NULL is a no-op. */
+void rtvla_vision_destroy(rtvla_vision_ctx *ctx);
+
 #ifdef __cplusplus
 }
 #endif
