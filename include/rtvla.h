@@ -1,6 +1,7 @@
 /*
- * rtvla.h — C ABI of librtvla.so: the π0.5 action-expert flow-matching denoise loop and the
- * Gemma-2B-shaped prefix pass that fills its KV cache, as hand-written CUDA for sm_100a.
+ * rtvla.h — C ABI of librtvla.so: the π0.5 action-expert flow-matching denoise loop, the
+ * Gemma-2B-shaped prefix pass that fills its KV cache, and the image front-end (SigLIP tower +
+ * projector) that produces the prefix's image embeddings, as hand-written CUDA for sm_100a.
  *
  * What the calls compute is defined by:
  *   [BLOG]  Realtime-VLA tech blog (blog.w4k4.me): "pi0.5 inference flow" (encoder phase run
