@@ -50,6 +50,27 @@ def test_host_side_argument_errors_without_gpu():
     assert e.value.name == "RTVLA_ERR_INVALID_ARG"
 
 
+def test_vision_host_side_argument_errors_without_gpu():
+    B.build()
+    lib = R.library()
+    with pytest.raises(R.RtvlaError) as e:
+        R.rtvla_vision_create({}, R.make_vision_config(n_layers=27))   # no weights
+    assert e.value.name == "RTVLA_ERR_INVALID_ARG"
+    cfg = R.make_vision_config(n_layers=2)
+    cfg.width = 1024
+    with pytest.raises(R.RtvlaError) as e:
+        R.rtvla_vision_create({}, cfg)                                 # a shape not built
+    assert e.value.name == "RTVLA_ERR_UNSUPPORTED"
+    cfg = R.make_vision_config(n_layers=2, max_images=0)
+    with pytest.raises(R.RtvlaError) as e:
+        R.rtvla_vision_create({}, cfg)
+    assert e.value.name == "RTVLA_ERR_INVALID_ARG"
+    assert R.STATUS[lib.rtvla_encode_images(None, None, 1, 1, None, 256, None)] == "RTVLA_ERR_INVALID_ARG"
+    assert R.STATUS[lib.rtvla_vision_sync_status(None, None)] == "RTVLA_ERR_INVALID_ARG"
+    assert lib.rtvla_vision_kernels_per_call(None, 1) == -1
+    R.rtvla_vision_destroy(0)
+
+
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(R, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(R, "_LIB", None)

@@ -53,3 +53,20 @@ def test_traffic_is_reported_only_for_unchanged_kernel_sources(monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 64)
     assert bench.measured_traffic(name, "persistent") is None
     assert bench.measured_traffic(name, "layered") is None
+
+
+def test_vision_bytes_and_flops():
+    # the SigLIP-So400m/14 matrices: patch 3*14*14 -> 1152, 27 x (q, k, v, o: 1152^2 each; fc1,
+    # fc2: 1152 x 4304 each), projector 1152 -> 2048
+    from synth import workloads as WL
+    mats = 588 * 1152 + 27 * (4 * 1152 ** 2 + 2 * 1152 * 4304) + 2048 * 1152
+    assert mats == 414_107_136
+    b, f = bench.vision_algorithmic(WL.VisionShape(), 2)
+    assert b == mats * 2 + 2 * 3 * 224 * 224 * 4 + 512 * 2048 * 2
+    assert f == 2 * 512 * mats + 27 * 2 * 16 * 4 * 256 * 256 * 72
+    assert abs(f / 1e9 - 440.35) < 0.01
+
+
+def test_prefill_kernel_count_matches_the_launch_list():
+    # 544-token prefill, 18 layers: 158 launches in the ncu launch list
+    assert bench.prefill_kernels(18) == 158
