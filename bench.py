@@ -7,6 +7,10 @@ resident in HBM.  Prints one JSON line (rank 0).  Multi-GPU runs are independent
 synchronize, and the time is the max over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--batch B]
+                  [--workload 2-view|1-view|3-view|e2e|stream|pi0|vision|pipeline] [--views V]
+
+Other workloads print their own line: the e2e prefill + denoise, the pi0 variant, the image
+encoder alone (vision) and full pi0 inference from camera views (pipeline).
 
 --impl reference times the fp64 CPU oracle (plain numpy) on the host cores: each step is
 one full 10-step loop of the same workload, after --warmup untimed loops.
