@@ -290,7 +290,10 @@ cudaError_t v_enqueue(rtvla_vision_ctx *c, int n_img, cudaStream_t st, float *tr
   const size_t hb = (size_t)M * VW * 4;
   VCK(launch_vis_embed(c->args, c->cols, c->h, c->table, n_img, st));
   VCK(gemm_launch(c->tm_wp, 0, c->xm_cols, M, VW, VKP, c->h, c->tmo_h, VW, nullptr, true, c->ctl, sm, st));
-  if (trace && cudaMemcpyAsync(trace, c->h, hb, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return cudaGetLastError();
+  if (trace) {
+    const cudaError_t e = cudaMemcpyAsync(trace, c->h, hb, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return e;
+  }
   for (int l = 0; l < L; ++l) {
     const int r0 = l * VROWS;
     VCK(launch_vis_ln(c->h, c->b_o + (size_t)l * VW, c->ln1_g + (size_t)l * VW, c->ln1_b + (size_t)l * VW, c->xn,
@@ -304,8 +307,10 @@ cudaError_t v_enqueue(rtvla_vision_ctx *c, int n_img, cudaStream_t st, float *tr
                     sm, st));
     VCK(launch_vis_gelu(c->acc, c->mb, M, VFP, st));
     VCK(gemm_launch(c->tm_wb, l * VW, c->xm_mb, M, VW, VFP, c->h, c->tmo_h, VW, nullptr, true, c->ctl, sm, st));
-    if (trace && cudaMemcpyAsync(trace + (size_t)(l + 1) * M * VW, c->h, hb, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-      return cudaGetLastError();
+    if (trace) {
+      const cudaError_t e = cudaMemcpyAsync(trace + (size_t)(l + 1) * M * VW, c->h, hb, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return e;
+    }
   }
   VCK(launch_vis_ln(c->h, nullptr, c->post_g, c->post_b, c->xn, c->acc, c->b_proj, VOUT, M, eps, st));
   VCK(gemm_launch(c->tm_wa, L * VROWS, c->xm_xn, M, VOUT, VW, c->acc, c->tmo_proj, VOUT, nullptr, true, c->ctl, sm, st));
