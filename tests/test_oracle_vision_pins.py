@@ -304,3 +304,16 @@ def test_images_recipe_is_uniform_in_range():
     w = WL.vision_weights(WL.VisionShape(n_layers=1))
     g = gen.bf16_to_f32(w["vis0.ln1_w"])
     assert abs(float(g.mean()) - 1.0) < 0.02 and 0.05 < float(g.std()) < 0.15
+
+
+def test_golden_regression_of_the_vision_oracle():
+    import importlib.util
+    import json
+    import os
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location("make_golden_vision", os.path.join(here, "make_golden_vision.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    stored = json.load(open(os.path.join(here, "tiny_vision_embeddings.json")))
+    expect = np.array([float.fromhex(x) for x in stored["embeddings"]]).reshape(stored["shape"])
+    np.testing.assert_allclose(mg.compute(), expect, rtol=1e-12, atol=1e-12)
