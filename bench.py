@@ -161,6 +161,17 @@ def vision_algorithmic(vcfg, n_img):
     return bytes_, flops
 
 
+def vision_config(vcfg, views, world):
+    """The `config` object of the image-encoder line, the same on both arms."""
+    return {"workload": f"SigLIP-So400m/14 shape, {views} x 224x224 views -> {views * vcfg.tokens} prefix embeddings",
+            "layers": vcfg.n_layers, "width": vcfg.width, "mlp": vcfg.mlp_dim, "heads": vcfg.n_heads,
+            "images": views, "tokens": views * vcfg.tokens, "parallelism": f"replicas{world}"}
+
+
+def vision_metric(views):
+    return f"image encoder latency ms ({views}-view, 27-layer SigLIP tower + projector)"
+
+
 def reduce_max(vals, device):
     """Each value's maximum over the ranks of the current process group (a replica job takes
     as long as its slowest rank); the values themselves without a group or with one rank."""
@@ -324,10 +335,12 @@ class OracleLoop:
 def run_reference(args, rank):
     if rank != 0:
         return
-    if args.workload in ("vision", "pipeline"):
-        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the denoise workloads; the "
-                          "image encoder's fp64 oracle is timed as the cpu_baseline of the repo arm's vision line"}),
-              flush=True)
+    if args.workload == "vision":
+        return run_reference_vision(args)
+    if args.workload == "pipeline":
+        print(json.dumps({"impl": "reference", "unavailable": "one step of the oracle chain (tower, 18-layer prefix "
+                          "pass, 10-step loop) takes minutes on the host cores; the vision and denoise workloads "
+                          "time its parts"}), flush=True)
         return
     wl = workload(args.batch, args.workload if args.workload not in ("e2e", "stream") else "2-view")
     loop = OracleLoop(wl)
@@ -346,6 +359,38 @@ def run_reference(args, rank):
                          "sample": f"{len(times)} full {wl.expert.n_steps}-step loops of the workload "
                                    f"(fp64 oracle), after {args.warmup} untimed"},
         "e2e": {"value": round(per_loop, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_vision(args):
+    """The fp64 image-encoder oracle on the host cores: each step encodes one of the --views
+    images (a bounded sample of the workload) and counts as views x its time."""
+    from oracle import vision as OV
+    from synth import workloads as WL
+    vcfg = WL.VisionShape()
+    V = args.views
+    W = WL.as_f32(WL.vision_weights(vcfg, tag="vision"))
+    imgs = WL.images(vcfg, V)
+    for i in range(args.warmup):
+        OV.encode_image(imgs[i % V], W, vcfg)
+    times = []
+    for i in range(max(1, args.steps)):
+        t0 = time.perf_counter()
+        OV.encode_image(imgs[i % V], W, vcfg)
+        times.append((time.perf_counter() - t0) * 1e3 * V)
+    per = statistics.mean(times)
+    line = {
+        "impl": "reference", "metric": vision_metric(V), "value": round(per, 1), "unit": "ms",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per, 1),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform [-1,1) f32 pixels)",
+        "config": vision_config(vcfg, V, args.gpus),
+        "engine": "oracle (fp64 numpy, host cores)",
+        "cpu_baseline": {"value": round(per, 1), "unit": "ms", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"each step one of the {V} images through the fp64 tower, times {V}, after "
+                                   f"{args.warmup} untimed"},
+        "e2e": {"value": round(per, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -857,14 +902,12 @@ def run_vision(args, rank, world, local_rank):
     t_roof = max(vb / (hbm * 1e9), vf / (bf16_pk * 1e12))
     achieved = vf / (ms * 1e-3) / 1e12
     line = {
-        "metric": f"image encoder latency ms ({V}-view, 27-layer SigLIP tower + projector)",
+        "metric": vision_metric(V),
         "value": round(ms, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform [-1,1) f32 pixels)",
-        "config": {"workload": f"SigLIP-So400m/14 shape, {V} x 224x224 views -> {P} prefix embeddings",
-                   "layers": vcfg.n_layers, "width": vcfg.width, "mlp": vcfg.mlp_dim, "heads": vcfg.n_heads,
-                   "images": V, "tokens": P, "parallelism": f"replicas{world}"},
+        "config": vision_config(vcfg, V, world),
         "l2": "flushed by a 256 MiB write between timed steps",
         "roofline": {"bound": "tensor", "kernel": "rtvla_encode_images (tcgen05 GEMMs + attention, one graph)",
                      "achieved": round(achieved, 1), "peak": bf16_pk, "unit": "TFLOP/s",

@@ -70,3 +70,19 @@ def test_vision_bytes_and_flops():
 def test_prefill_kernel_count_matches_the_launch_list():
     # 544-token prefill, 18 layers: 158 launches in the ncu launch list
     assert bench.prefill_kernels(18) == 158
+
+
+def test_vision_reference_arm_prints_the_arms_metric_and_config(monkeypatch, capsys):
+    import functools
+    import json
+    from types import SimpleNamespace
+
+    from synth import workloads as WL
+    monkeypatch.setattr(WL, "VisionShape", functools.partial(WL.VisionShape, n_layers=1))   # a short tower
+    args = SimpleNamespace(workload="vision", views=2, steps=1, warmup=0, gpus=1, batch=1)
+    bench.run_reference(args, 0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.vision_metric(2)
+    assert line["config"] == bench.vision_config(WL.VisionShape(), 2, 1)
+    assert line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
